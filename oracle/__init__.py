@@ -1,0 +1,142 @@
+"""fp64 CPU oracle for hybrid sliding-window attention (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` and
+``--impl reference`` legs of ``bench.py`` may import this package. The product
+path (``hybrid_sliding_window_swa_b200``) never imports it and shares no code
+with it. The arithmetic lives in ``oracle.c`` (plain C, fp64); this module only
+builds it with gcc and marshals numpy/torch arrays through ctypes.
+
+Every function here restates a passage of the source pages; see ``oracle.h``
+for the citations and the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (host code only)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
+            os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "oracle.h"))):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        i64, i32, p = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+        L.orc_mask_count.restype = i64
+        L.orc_mask_count.argtypes = [i64, i64]
+        L.orc_attention.restype = i32
+        L.orc_attention.argtypes = [p, p, i64, i32, p, p, i64, i64, i32, i32, i64, p, i32]
+        L.orc_window_safe_len.restype = i32
+        L.orc_window_safe_len.argtypes = [p, p, p, ctypes.c_int32, i64, p]
+        L.orc_ring_trace.restype = i32
+        L.orc_ring_trace.argtypes = [i64, i64, p]
+        L.orc_kv_bytes.restype = i64
+        L.orc_kv_bytes.argtypes = [i64, i64, i64, i64, i64]
+        L.orc_hybrid_kv_ratio.restype = ctypes.c_double
+        L.orc_hybrid_kv_ratio.argtypes = [i64, i64, i64, i64]
+        _lib = L
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 data (torch bf16 tensor or uint16/int16 numpy array) -> contiguous uint16 numpy."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(x)
+    assert a.dtype in (np.uint16, np.int16)
+    return a.view(np.uint16)
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def mask_count(n: int, window: int) -> int:
+    """Pairs (i, j) with j in W(i) for i < n (window 0 = full causal)."""
+    return int(_load().orc_mask_count(n, window))
+
+
+def attention(q, q_pos, k, v, window: int, key_base: int = 0, n_threads: int | None = None) -> np.ndarray:
+    """fp64 attention rows.
+
+    q: [n_rows, Hq, d] bf16; q_pos: [n_rows] absolute positions;
+    k, v: [n_keys, Hkv, d] bf16 holding positions key_base .. key_base+n_keys-1;
+    window >= 1 (sliding window) or 0 (full causal). Returns [n_rows, Hq, d] float64.
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    assert qb.ndim == 3 and kb.ndim == 3 and vb.shape == kb.shape
+    n_rows, hq, d = qb.shape
+    n_keys, hkv, d2 = kb.shape
+    assert d == d2
+    pos = np.ascontiguousarray(np.asarray(q_pos, dtype=np.int64))
+    assert pos.shape == (n_rows,)
+    out = np.empty((n_rows, hq, d), dtype=np.float64)
+    rc = _load().orc_attention(qb.ctypes.data, pos.ctypes.data, n_rows, hq, kb.ctypes.data,
+                               vb.ctypes.data, key_base, n_keys, hkv, d, window,
+                               out.ctypes.data, n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle attention: a needed key position is outside the given keys")
+    return out
+
+
+def window_safe_len(match_len, cached_len, slot_valid, window: int) -> np.ndarray:
+    """Window-safe prefix-match length per request, by definition (int64)."""
+    m = np.ascontiguousarray(np.asarray(match_len, dtype=np.int64))
+    c = np.ascontiguousarray(np.asarray(cached_len, dtype=np.int64))
+    words = (window + 31) // 32
+    sv = np.ascontiguousarray(np.asarray(slot_valid, dtype=np.uint32)).reshape(-1)
+    assert m.shape == c.shape and sv.size == m.size * words
+    out = np.empty(m.shape, dtype=np.int64)
+    rc = _load().orc_window_safe_len(m.ctypes.data, c.ctypes.data, sv.ctypes.data, window,
+                                     m.size, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle window_safe_len: bad arguments")
+    return out
+
+
+def ring_trace(n_appended: int, w: int) -> np.ndarray:
+    """Position held by each of the w ring slots after appending positions 0..n_appended-1."""
+    out = np.empty(w, dtype=np.int64)
+    assert _load().orc_ring_trace(n_appended, w, out.ctypes.data) == 0
+    return out
+
+
+def kv_bytes(layers: int, kv_heads: int, tokens: int, head_dim: int, elem_bytes: int = 2) -> int:
+    return int(_load().orc_kv_bytes(layers, kv_heads, tokens, head_dim, elem_bytes))
+
+
+def hybrid_kv_ratio(n_swa: int, n_full: int, window: int, n_tokens: int) -> float:
+    return float(_load().orc_hybrid_kv_ratio(n_swa, n_full, window, n_tokens))
+
+
+def pool_bytes(n_swa_layers: int, n_full_layers: int, window: int, n_kv_heads: int,
+               head_dim: int, page_size: int, max_seqs: int, pages_per_full_layer: int,
+               elem_bytes: int = 2) -> tuple[int, int]:
+    """(SWA ring bytes, full paged-pool bytes) of the dual pool, from the KV-bytes formula:
+    each sequence keeps W token-slots per SWA layer; each full layer keeps
+    pages * page_size token-slots."""
+    swa = kv_bytes(n_swa_layers, n_kv_heads, window * max_seqs, head_dim, elem_bytes)
+    full = kv_bytes(n_full_layers, n_kv_heads, pages_per_full_layer * page_size, head_dim, elem_bytes)
+    return swa, full
