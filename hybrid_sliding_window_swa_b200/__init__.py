@@ -1,0 +1,278 @@
+"""hybrid_sliding_window_swa_b200 -- hybrid sliding-window attention on NVIDIA B200.
+
+Thin Python binding over ``libhswa.so`` (C ABI in ``include/hswa.h``). Every function
+here has the name of the C entry point it calls and only marshals arguments
+(torch tensors -> device pointers, the current CUDA stream); all computation runs
+in the library's sm_100a kernels. There is no fallback: if the library is missing
+or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhswa.so")
+
+HSWA_OK = 0
+HSWA_ERR_INVALID_ARG = -1
+HSWA_ERR_UNSUPPORTED_SHAPE = -2
+HSWA_ERR_OUT_OF_MEMORY = -3
+HSWA_ERR_CUDA = -4
+HSWA_ERR_TIMEOUT = -5
+HSWA_ERR_DEVICE_BOUNDS = -6
+
+EXPORTED = [
+    "kv_pool_layout", "kv_pool_create", "kv_pool_destroy", "kv_pool_append",
+    "swa_prefill_fwd", "full_prefill_fwd", "hybrid_decode_workspace_size", "hybrid_decode_fwd",
+    "window_safe_len", "hswa_pool_check_error", "hswa_last_error",
+]
+
+
+class HswaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"hswa error {code}: {msg}")
+        self.code = code
+
+
+class PoolDescC(ctypes.Structure):
+    _fields_ = [
+        ("n_swa_layers", ctypes.c_int32), ("n_full_layers", ctypes.c_int32), ("window", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("max_seqs", ctypes.c_int32), ("reserved", ctypes.c_int32), ("pages_per_full_layer", ctypes.c_int64),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Load libhswa.so (raises if it is absent: there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libhswa.so not found at {path}; build it with "
+                          f"`python -m hybrid_sliding_window_swa_b200._build`")
+    L = ctypes.CDLL(path)
+    p, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "kv_pool_layout": [ctypes.POINTER(PoolDescC), ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)],
+        "kv_pool_create": [ctypes.POINTER(PoolDescC), p, sz, ctypes.POINTER(p)],
+        "kv_pool_destroy": [p],
+        "kv_pool_append": [p, i32, i32, p, p, i32, p, p, p, i32, p],
+        "swa_prefill_fwd": [p, i32, p, p, p, p, i32, i32, p, p, i32, p],
+        "full_prefill_fwd": [p, i32, p, p, i32, i32, p, p, i32, i32, p],
+        "hybrid_decode_workspace_size": [p, i32, i32, i32, i64, ctypes.POINTER(sz)],
+        "hybrid_decode_fwd": [p, i32, p, p, p, p, i32, i32, p, i64, p, p, i32, i32, p, sz, p],
+        "window_safe_len": [p, p, p, ctypes.c_int32, ctypes.c_int32, p, p],
+        "hswa_pool_check_error": [p, ctypes.POINTER(ctypes.c_int)],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    L.hswa_last_error.argtypes = []
+    L.hswa_last_error.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != HSWA_OK:
+        msg = load_library().hswa_last_error().decode(errors="replace")
+        raise HswaError(rc, msg)
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name: str = "tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+@dataclass(frozen=True)
+class PoolDesc:
+    n_swa_layers: int
+    n_full_layers: int
+    window: int
+    n_kv_heads: int
+    head_dim: int
+    max_seqs: int
+    pages_per_full_layer: int
+    page_size: int = 64
+
+    def c(self) -> PoolDescC:
+        return PoolDescC(self.n_swa_layers, self.n_full_layers, self.window, self.n_kv_heads, self.head_dim,
+                         self.page_size, self.max_seqs, 0, self.pages_per_full_layer)
+
+
+def kv_pool_layout(desc: PoolDesc) -> tuple[int, int, int]:
+    """(bytes_total, bytes_swa, bytes_full) of the dual pool."""
+    L = load_library()
+    t, s, f = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    d = desc.c()
+    _check(L.kv_pool_layout(ctypes.byref(d), ctypes.byref(t), ctypes.byref(s), ctypes.byref(f)))
+    return t.value, s.value, f.value
+
+
+class KVPool:
+    """A dual-pool KV cache carved out of one caller-owned torch uint8 CUDA buffer."""
+
+    def __init__(self, desc: PoolDesc, memory: torch.Tensor, handle):
+        self.desc = desc
+        self.memory = memory
+        self.handle = handle
+
+    def _views(self):
+        d = self.desc
+        _, swa, _full = kv_pool_layout(d)
+        ring_half = d.max_seqs * d.n_swa_layers * d.n_kv_heads * d.window * d.head_dim
+        page_half = d.n_full_layers * d.pages_per_full_layer * d.n_kv_heads * d.page_size * d.head_dim
+        mem = self.memory
+        ring = mem[: 4 * ring_half].view(torch.bfloat16).view(2, d.max_seqs, d.n_swa_layers, d.n_kv_heads,
+                                                               d.window, d.head_dim)
+        pages = mem[swa: swa + 4 * page_half].view(torch.bfloat16).view(
+            2, d.n_full_layers, d.pages_per_full_layer, d.n_kv_heads, d.page_size, d.head_dim)
+        return ring, pages
+
+    @property
+    def ring(self) -> torch.Tensor:
+        """[2 (K,V)][max_seqs][n_swa_layers][Hkv][W][d] view of the rolling buffers."""
+        return self._views()[0]
+
+    @property
+    def pages(self) -> torch.Tensor:
+        """[2 (K,V)][n_full_layers][pages][Hkv][page_size][d] view of the paged pool."""
+        return self._views()[1]
+
+    def destroy(self):
+        if self.handle is not None:
+            load_library().kv_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def kv_pool_create(desc: PoolDesc, memory: torch.Tensor | None = None, device=None) -> KVPool:
+    """Carve a pool from ``memory`` (uint8 CUDA tensor of >= bytes_total) or allocate one with torch."""
+    L = load_library()
+    total, _, _ = kv_pool_layout(desc)
+    if memory is None:
+        memory = torch.empty(total, dtype=torch.uint8, device=device or "cuda")
+    _ptr(memory, torch.uint8, "memory")
+    h = ctypes.c_void_p()
+    d = desc.c()
+    _check(L.kv_pool_create(ctypes.byref(d), ctypes.c_void_p(memory.data_ptr()), memory.numel(), ctypes.byref(h)))
+    return KVPool(desc, memory, h)
+
+
+def kv_pool_destroy(pool: KVPool):
+    pool.destroy()
+
+
+def kv_pool_append(pool: KVPool, layer: int, k: torch.Tensor, v: torch.Tensor, start_pos: torch.Tensor,
+                   seq_ids: torch.Tensor | None = None, page_table: torch.Tensor | None = None, stream=None):
+    """Commit k, v [n_seqs, n_tok, Hkv, d] at positions start_pos[b] + t of layer ``layer``."""
+    n_seqs, n_tok = k.shape[0], k.shape[1]
+    pt_stride = page_table.shape[1] if page_table is not None else 0
+    _check(load_library().kv_pool_append(
+        pool.handle, layer, n_seqs, _ptr(seq_ids, torch.int32, "seq_ids"), _ptr(start_pos, torch.int64, "start_pos"),
+        n_tok, _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+        _ptr(page_table, torch.int32, "page_table"), pt_stride, _stream(stream)))
+
+
+def swa_prefill_fwd(pool: KVPool, layer: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    o: torch.Tensor | None = None, start_pos: torch.Tensor | None = None,
+                    seq_ids: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Sliding-window attention of a chunk: q [B, n_q, Hq, d], k/v [B, n_q, Hkv, d] -> o like q."""
+    B, n_q, hq, _ = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    _check(load_library().swa_prefill_fwd(
+        pool.handle, layer, _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+        _ptr(v, torch.bfloat16, "v"), _ptr(o, torch.bfloat16, "o"), B, n_q,
+        _ptr(start_pos, torch.int64, "start_pos"), _ptr(seq_ids, torch.int32, "seq_ids"), hq, _stream(stream)))
+    return o
+
+
+def full_prefill_fwd(pool: KVPool, layer: int, q: torch.Tensor, page_table: torch.Tensor,
+                     o: torch.Tensor | None = None, start_pos: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Full causal attention of a chunk over the paged pool (the chunk must be appended first)."""
+    B, n_q, hq, _ = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    _check(load_library().full_prefill_fwd(
+        pool.handle, layer, _ptr(q, torch.bfloat16, "q"), _ptr(o, torch.bfloat16, "o"), B, n_q,
+        _ptr(start_pos, torch.int64, "start_pos"), _ptr(page_table, torch.int32, "page_table"),
+        page_table.shape[1], hq, _stream(stream)))
+    return o
+
+
+def hybrid_decode_workspace_size(pool: KVPool, n_seqs: int, n_q_per_seq: int, n_q_heads: int,
+                                 max_ctx_len: int) -> int:
+    out = ctypes.c_size_t()
+    _check(load_library().hybrid_decode_workspace_size(pool.handle, n_seqs, n_q_per_seq, n_q_heads,
+                                                       max_ctx_len, ctypes.byref(out)))
+    return out.value
+
+
+def hybrid_decode_fwd(pool: KVPool, layer: int, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                      ctx_len: torch.Tensor, max_ctx_len: int, workspace: torch.Tensor,
+                      seq_ids: torch.Tensor | None = None, page_table: torch.Tensor | None = None,
+                      o: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One decode step: q [n_seqs, n_qt, Hq, d], k_new/v_new [n_seqs, n_qt, Hkv, d] -> o like q."""
+    n_seqs, n_qt, hq, _ = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    pt_stride = page_table.shape[1] if page_table is not None else 0
+    _check(load_library().hybrid_decode_fwd(
+        pool.handle, layer, _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(o, torch.bfloat16, "o"), n_seqs, n_qt,
+        _ptr(ctx_len, torch.int64, "ctx_len"), max_ctx_len, _ptr(seq_ids, torch.int32, "seq_ids"),
+        _ptr(page_table, torch.int32, "page_table"), pt_stride, hq, _ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)))
+    return o
+
+
+def window_safe_len(match_len: torch.Tensor, cached_len: torch.Tensor, slot_valid: torch.Tensor, window: int,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Window-safe prefix-match length per request (int64, exact)."""
+    n = match_len.numel()
+    if out is None:
+        out = torch.empty(n, dtype=torch.int64, device=match_len.device)
+    sv = slot_valid.view(torch.int32) if slot_valid.dtype == torch.uint32 else slot_valid
+    _check(load_library().window_safe_len(
+        _ptr(match_len, torch.int64, "match_len"), _ptr(cached_len, torch.int64, "cached_len"),
+        _ptr(sv, torch.int32, "slot_valid"), window, n, _ptr(out, torch.int64, "out"), _stream(stream)))
+    return out
+
+
+def hswa_pool_check_error(pool: KVPool) -> int:
+    """Synchronise and return (then clear) the pool's device error code (0 = none)."""
+    code = ctypes.c_int()
+    _check(load_library().hswa_pool_check_error(pool.handle, ctypes.byref(code)))
+    return code.value
+
+
+def hswa_last_error() -> str:
+    return load_library().hswa_last_error().decode(errors="replace")

@@ -1,0 +1,632 @@
+// decode.cu -- one decode step of hybrid sliding-window attention, split over the KV
+// sequence ("split-KV"), plus the log-sum-exp merge of the splits.
+//
+// Each sequence brings n_qt new query tokens at positions L .. L+n_qt-1 (one token and
+// its multi-token-prediction drafts; "MiMo v2.5 inference optimisation", sections
+// "architecture" and "KV cache redesign"). Draft t attends the cached keys in its window
+// plus new tokens 0..t. Sliding-window layers read cached keys from the rolling buffer
+// (slot = pos mod W, "Sliding Window Attention (SWA) no riron to jisso", section
+// "Rolling Buffer KV Cache", eq. (7)); full layers read them through the page table.
+//
+// Work item = (sequence s, split c, KV head g): keys [klo + c*SPLIT, klo + (c+1)*SPLIT)
+// of the cached range, plus the new tokens in the sequence's last split. The rows of an
+// item are the n_qt * G query rows (token t, query head g*G + hh) that share KV head g,
+// so every K/V byte is read from HBM once per step. A CTA of 4 warps streams 64-key
+// blocks of K and V through a 3-stage cp.async pipeline; each warp takes 16 keys of a
+// block, computes S = Q K^T and O += P V with mma.sync (bf16 in, fp32 accumulate), and
+// keeps its own online-softmax state; the 4 warp states are merged through shared
+// memory at the end of the item. Items with one split write the output directly; the
+// others write (m, l, O) partials that merge_kernel combines:
+//   o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hswa {
+
+namespace {
+
+constexpr int DEC_THREADS = 128;
+constexpr int KB = 64;          // keys per block
+constexpr int NST = 3;          // pipeline stages
+constexpr int SPLIT = 4096;     // cached keys per split (multiple of KB)
+
+struct WsHeader {
+  int counter;
+  int total_items;
+  int pad[62];
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t prefix_off, part_off, part_bytes_per_item, bytes;
+  __host__ __device__ WsLayout(int n_seqs, int rows, int d, int64_t max_items) {
+    prefix_off = sizeof(WsHeader);
+    part_off = align256(prefix_off + sizeof(int) * (size_t)(n_seqs + 1));
+    part_bytes_per_item = (size_t)rows * (d + 2) * sizeof(float);
+    bytes = part_off + part_bytes_per_item * (size_t)max_items;
+  }
+};
+
+struct DecParams {
+  int n_seqs, n_qt, Hq, Hkv, G, R, window;
+  const uint16_t* q;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* o;
+  const int64_t* ctx_len;
+  int64_t max_ctx_len;
+  const int32_t* seq_ids;
+  const int32_t* page_table;
+  int pt_stride;
+  const uint16_t* src_k;  // ring or page base of the layer
+  const uint16_t* src_v;
+  int n_swa, ring_layer, max_seqs;
+  int full_layer;
+  int64_t pages;
+  float scale_log2;
+  uint8_t* ws;
+  size_t part_off, part_bytes;
+  int* err;
+};
+
+__device__ __forceinline__ int64_t dec_klo(const DecParams& p, int64_t L) {
+  if (p.window <= 0) return 0;
+  const int64_t lo = L - p.window + 1;
+  return lo > 0 ? lo : 0;
+}
+
+__device__ __forceinline__ int n_splits(const DecParams& p, int64_t L) {
+  const int64_t cached = L - dec_klo(p, L);
+  const int64_t n = (cached + SPLIT - 1) / SPLIT;
+  return n < 1 ? 1 : (int)n;
+}
+
+__device__ __forceinline__ int64_t safe_len(const DecParams& p, int s) {
+  int64_t L = p.ctx_len[s];
+  if (L < 0 || L > p.max_ctx_len) {
+    record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+    L = 0;
+  }
+  return L;
+}
+
+// Prefix sums of the split counts; resets the work counter.
+__global__ void __launch_bounds__(1024) plan_kernel(DecParams p) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
+  int* prefix = reinterpret_cast<int*>(p.ws + sizeof(WsHeader));
+  __shared__ int carry;
+  __shared__ int warp_sums[32];
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < p.n_seqs; base += 1024) {
+    const int s = base + threadIdx.x;
+    int v = s < p.n_seqs ? n_splits(p, safe_len(p, s)) : 0;
+    // block-wide inclusive scan
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += y;
+    }
+    if (lane == 31) warp_sums[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int ws = warp_sums[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, ws, d);
+        if (lane >= d) ws += y;
+      }
+      warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    const int incl = x + (w > 0 ? warp_sums[w - 1] : 0) + carry;
+    if (s < p.n_seqs) prefix[s + 1] = incl;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    prefix[0] = 0;
+    hdr->total_items = carry * p.Hkv;
+    hdr->counter = 0;
+  }
+}
+
+// ---------------------------------------------------------------- mma.sync helpers
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// byte offset of 16-byte chunk `c` of row `r` in a [rows][D] bf16 tile, XOR-swizzled
+template <int D>
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return (uint32_t)(r * (D * 2) + ((c ^ (r & 7)) << 4));
+}
+
+template <int D, int MT>
+struct DecSmem {
+  static constexpr int ROWS = 16 * MT;
+  static constexpr int TILE = KB * D * 2;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + NST * TILE;
+  static constexpr int Q_OFF = V_OFF + NST * TILE;
+  static constexpr int MISC_OFF = Q_OFF + ROWS * D * 2;
+  // merge area aliases the K stages (idle while merging)
+  static constexpr int ACC_OFF = 0;
+  static constexpr int BYTES = MISC_OFF + 4 * ROWS * 4 * 2 + ROWS * 4 * 2 + 64;
+  static_assert(ROWS * D * 4 <= NST * TILE, "merge buffer must fit in the K stages");
+};
+
+template <int D, int MT>
+__global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
+  using SM = DecSmem<D, MT>;
+  constexpr int ROWS = SM::ROWS;
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t smem[];
+  float* m_w = reinterpret_cast<float*>(smem + SM::MISC_OFF);   // [4][ROWS]
+  float* l_w = m_w + 4 * ROWS;                                  // [4][ROWS]
+  float* m_all = l_w + 4 * ROWS;                                // [ROWS]
+  float* l_all = m_all + ROWS;                                  // [ROWS]
+  int* item_slot = reinterpret_cast<int*>(l_all + ROWS);
+  const uint32_t s_base = smem_u32(smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
+  const int* prefix = reinterpret_cast<const int*>(p.ws + sizeof(WsHeader));
+
+  if (read_error(p.err) != 0) return;
+
+  for (;;) {
+    if (tid == 0) *item_slot = atomicAdd(&hdr->counter, 1);
+    __syncthreads();
+    const int item = *item_slot;
+    __syncthreads();
+    if (item >= hdr->total_items) break;
+    const int g = item % p.Hkv;
+    const int sc = item / p.Hkv;
+    // sequence s: prefix[s] <= sc < prefix[s + 1]
+    int lo = 0, hi = p.n_seqs;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= sc) lo = mid; else hi = mid;
+    }
+    const int s = lo;
+    const int c = sc - prefix[s];
+    const int nsp = prefix[s + 1] - prefix[s];
+    const bool last = c == nsp - 1;
+    const int64_t L = safe_len(p, s);
+    const int64_t klo = dec_klo(p, L);
+    const int64_t a = klo + (int64_t)c * SPLIT;
+    const int64_t b = (a + SPLIT < L) ? a + SPLIT : L;
+    const int n_cached_blk = (int)((b - a + KB - 1) / KB);
+    const int n_blk = n_cached_blk + (last ? 1 : 0);
+    int64_t ring_row = 0;
+    if (p.window > 0) {
+      const int seq = p.seq_ids[s];
+      if (seq < 0 || seq >= p.max_seqs) {
+        record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+        ring_row = -1;
+      } else {
+        ring_row = (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + g) * p.window;
+      }
+    }
+
+    // ---- stage Q rows (row = t * G + hh) into shared memory, zero rows >= R
+    for (int idx = tid; idx < ROWS * CH; idx += DEC_THREADS) {
+      const int r = idx / CH, ch = idx % CH;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (r < p.R) {
+        const int t = r / p.G, hh = r % p.G;
+        const uint16_t* src = p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
+        val = *reinterpret_cast<const uint4*>(src);
+      }
+      *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, ch)) = val;
+    }
+
+    // ---- block loader: block kb2 of this item into stage st
+    auto load_block = [&](int kb2, int st) {
+      for (int idx = tid; idx < KB * CH; idx += DEC_THREADS) {
+        const int r = idx / CH, ch = idx % CH;
+        const uint16_t* sk = p.src_k;  // any valid address for zero-fill
+        const uint16_t* sv = p.src_v;
+        uint32_t bytes = 0;
+        if (kb2 < n_cached_blk) {
+          const int64_t pos = a + (int64_t)kb2 * KB + r;
+          if (pos < b) {
+            int64_t row = -1;
+            if (p.window > 0) {
+              if (ring_row >= 0) row = ring_row + pos % p.window;
+            } else {
+              const int64_t lp = pos / 64;
+              const int32_t page = lp < p.pt_stride ? p.page_table[(int64_t)s * p.pt_stride + lp] : -1;
+              if (page < 0 || page >= p.pages) {
+                record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+              } else {
+                row = (((int64_t)p.full_layer * p.pages + page) * p.Hkv + g) * 64 + pos % 64;
+              }
+            }
+            if (row >= 0) {
+              sk = p.src_k + row * D + ch * 8;
+              sv = p.src_v + row * D + ch * 8;
+              bytes = 16;
+            }
+          }
+        } else if (r < p.n_qt) {
+          const int64_t row = ((int64_t)s * p.n_qt + r) * p.Hkv + g;
+          sk = p.k_new + row * D + ch * 8;
+          sv = p.v_new + row * D + ch * 8;
+          bytes = 16;
+        }
+        cp_async_16(s_base + SM::K_OFF + st * SM::TILE + sw_off<D>(r, ch), sk, bytes);
+        cp_async_16(s_base + SM::V_OFF + st * SM::TILE + sw_off<D>(r, ch), sv, bytes);
+      }
+    };
+
+#pragma unroll
+    for (int st = 0; st < NST - 1; ++st) {
+      if (st < n_blk) load_block(st, st);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+
+    // per-thread row state: rows (mt*16 + lane/4) and (+8)
+    float o_acc[MT][D / 8][4];
+    float m_r[MT][2], l_r[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      m_r[mt][0] = m_r[mt][1] = -INFINITY;
+      l_r[mt][0] = l_r[mt][1] = 0.f;
+#pragma unroll
+      for (int nd = 0; nd < D / 8; ++nd) o_acc[mt][nd][0] = o_acc[mt][nd][1] = o_acc[mt][nd][2] = o_acc[mt][nd][3] = 0.f;
+    }
+    // per-row query token t and window start, for the two rows of each M tile
+    int64_t row_pos[MT][2], row_lo[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = mt * 16 + (lane >> 2) + hf * 8;
+        const int t = r < p.R ? r / p.G : 0;
+        row_pos[mt][hf] = L + t;
+        int64_t lo2 = 0;
+        if (p.window > 0) {
+          lo2 = L + t - p.window + 1;
+          if (lo2 < 0) lo2 = 0;
+        }
+        row_lo[mt][hf] = r < p.R ? lo2 : INT64_MAX;  // padding rows see nothing
+      }
+
+    for (int kb2 = 0; kb2 < n_blk; ++kb2) {
+      {
+        const int nxt = kb2 + NST - 1;
+        if (nxt < n_blk) load_block(nxt, nxt % NST);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      asm volatile("cp.async.wait_group %0;" ::"n"(NST - 1) : "memory");
+      __syncthreads();
+      const int st = kb2 % NST;
+      const uint32_t kt = s_base + SM::K_OFF + st * SM::TILE;
+      const uint32_t vt = s_base + SM::V_OFF + st * SM::TILE;
+      const uint32_t qt = s_base + SM::Q_OFF;
+      const int key0 = warp * 16;  // this warp's 16 keys of the block
+
+      // S = Q K^T for ROWS x 16 keys
+      float sacc[MT][2][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) sacc[mt][nt][0] = sacc[mt][nt][1] = sacc[mt][nt][2] = sacc[mt][nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        {
+          const int mi = lane >> 3;
+          const int key = key0 + (mi >> 1) * 8 + (lane & 7);
+          ldsm_x4(kt + sw_off<D>(key, kk * 2 + (mi & 1)), b0, b1, b2, b3);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          const int mi = lane >> 3;
+          const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
+          ldsm_x4(qt + sw_off<D>(row, kk * 2 + (mi >> 1)), a0, a1, a2, a3);
+          mma_bf16(sacc[mt][0], a0, a1, a2, a3, b0, b1);
+          mma_bf16(sacc[mt][1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+      // mask + online softmax (exp2 domain)
+      int64_t kpos_base;
+      bool is_new = kb2 >= n_cached_blk;
+      kpos_base = is_new ? L : a + (int64_t)kb2 * KB;
+      uint32_t pa[MT][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int kcol = key0 + nt * 8 + (lane & 3) * 2 + e;
+              const int64_t pos = kpos_base + kcol;
+              bool ok;
+              if (is_new) ok = kcol < p.n_qt && pos <= row_pos[mt][hf] && pos >= row_lo[mt][hf];
+              else ok = pos < b && pos >= row_lo[mt][hf];
+              const float sv = sacc[mt][nt][hf * 2 + e];
+              v[nt * 2 + e] = ok ? sv * p.scale_log2 : -INFINITY;
+            }
+          float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float m_new = fmaxf(m_r[mt][hf], mx);
+          const float moff = m_new == -INFINITY ? 0.f : m_new;
+          const float alpha = ex2_approx(m_r[mt][hf] - moff);  // 0 when the old max is -inf
+          m_r[mt][hf] = m_new;
+          float pv[4];
+          float rs = 0.f;
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            pv[x] = ex2_approx(v[x] - moff);
+            rs += pv[x];
+          }
+          l_r[mt][hf] = l_r[mt][hf] * alpha + rs;
+#pragma unroll
+          for (int nd = 0; nd < D / 8; ++nd) {
+            o_acc[mt][nd][hf * 2 + 0] *= alpha;
+            o_acc[mt][nd][hf * 2 + 1] *= alpha;
+          }
+          // A fragment of P (16 rows x 16 keys): a0/a1 = keys 0-7 (rows r, r+8), a2/a3 = keys 8-15
+          pa[mt][hf + 0] = pack_bf16x2(pv[0], pv[1]);
+          pa[mt][hf + 2] = pack_bf16x2(pv[2], pv[3]);
+        }
+      }
+      // O += P V  (16 keys x D)
+#pragma unroll
+      for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+        uint32_t b0, b1, b2, b3;
+        const int mi = lane >> 3;
+        const int key = key0 + (mi & 1) * 8 + (lane & 7);
+        ldsm_x4_t(vt + sw_off<D>(key, nd2 * 2 + (mi >> 1)), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          mma_bf16(o_acc[mt][nd2 * 2 + 0], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b0, b1);
+          mma_bf16(o_acc[mt][nd2 * 2 + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b2, b3);
+        }
+      }
+      __syncthreads();  // the stage may be overwritten by the next iteration's loads
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+    // ---- merge the 4 warps' states
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float lsum = l_r[mt][hf];
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        l_r[mt][hf] = lsum;
+        if ((lane & 3) == 0) {
+          const int r = mt * 16 + (lane >> 2) + hf * 8;
+          m_w[warp * ROWS + r] = m_r[mt][hf];
+          l_w[warp * ROWS + r] = lsum;
+        }
+      }
+    float* acc = reinterpret_cast<float*>(smem + SM::ACC_OFF);
+    __syncthreads();
+    for (int idx = tid; idx < ROWS * D; idx += DEC_THREADS) acc[idx] = 0.f;
+    for (int r = tid; r < ROWS; r += DEC_THREADS) {
+      float M = -INFINITY;
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, m_w[w * ROWS + r]);
+      const float Mo = M == -INFINITY ? 0.f : M;
+      float Ls = 0.f;
+      for (int w = 0; w < 4; ++w) Ls += l_w[w * ROWS + r] * ex2_approx(m_w[w * ROWS + r] - Mo);
+      m_all[r] = M;
+      l_all[r] = Ls;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = mt * 16 + (lane >> 2) + hf * 8;
+        const float Mo = m_all[r] == -INFINITY ? 0.f : m_all[r];
+        const float f = ex2_approx(m_r[mt][hf] - Mo);
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd) {
+          const int col = nd * 8 + (lane & 3) * 2;
+          atomicAdd(&acc[r * D + col], o_acc[mt][nd][hf * 2 + 0] * f);
+          atomicAdd(&acc[r * D + col + 1], o_acc[mt][nd][hf * 2 + 1] * f);
+        }
+      }
+    __syncthreads();
+    if (nsp == 1) {
+      // single split: normalise and write bf16 output rows
+      for (int idx = tid; idx < p.R * (D / 8); idx += DEC_THREADS) {
+        const int r = idx / (D / 8), ch = idx % (D / 8);
+        const float inv = 1.f / l_all[r];
+        const float* src = acc + r * D + ch * 8;
+        uint4 pk;
+        pk.x = pack_bf16x2(src[0] * inv, src[1] * inv);
+        pk.y = pack_bf16x2(src[2] * inv, src[3] * inv);
+        pk.z = pack_bf16x2(src[4] * inv, src[5] * inv);
+        pk.w = pack_bf16x2(src[6] * inv, src[7] * inv);
+        const int t = r / p.G, hh = r % p.G;
+        uint16_t* dst = p.o + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
+        *reinterpret_cast<uint4*>(dst) = pk;
+      }
+    } else {
+      float* part = reinterpret_cast<float*>(p.ws + p.part_off + (size_t)item * p.part_bytes);
+      for (int idx = tid; idx < p.R * D; idx += DEC_THREADS) part[idx] = acc[idx];
+      for (int r = tid; r < p.R; r += DEC_THREADS) {
+        part[p.R * D + r] = m_all[r];
+        part[p.R * D + p.R + r] = l_all[r];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// One CTA per (sequence, KV head) with more than one split.
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
+  const int g = blockIdx.x % p.Hkv;
+  const int s = blockIdx.x / p.Hkv;
+  const int* prefix = reinterpret_cast<const int*>(p.ws + sizeof(WsHeader));
+  const int c0 = prefix[s];
+  const int nsp = prefix[s + 1] - c0;
+  if (nsp <= 1) return;
+  extern __shared__ float msh[];  // [nsp][R] scale factors, then [R] inverse denominators
+  float* fac = msh;
+  float* inv = msh + (size_t)nsp * p.R;
+  for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+    float M = -INFINITY;
+    for (int c = 0; c < nsp; ++c) {
+      const float* part =
+          reinterpret_cast<const float*>(p.ws + p.part_off + (size_t)((c0 + c) * p.Hkv + g) * p.part_bytes);
+      M = fmaxf(M, part[p.R * D + r]);
+    }
+    const float Mo = M == -INFINITY ? 0.f : M;
+    float den = 0.f;
+    for (int c = 0; c < nsp; ++c) {
+      const float* part =
+          reinterpret_cast<const float*>(p.ws + p.part_off + (size_t)((c0 + c) * p.Hkv + g) * p.part_bytes);
+      const float f = ex2_approx(part[p.R * D + r] - Mo);
+      fac[c * p.R + r] = f;
+      den += f * part[p.R * D + p.R + r];
+    }
+    inv[r] = 1.f / den;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < p.R * (D / 2); idx += blockDim.x) {
+    const int r = idx / (D / 2), col = (idx % (D / 2)) * 2;
+    float x0 = 0.f, x1 = 0.f;
+    for (int c = 0; c < nsp; ++c) {
+      const float* part =
+          reinterpret_cast<const float*>(p.ws + p.part_off + (size_t)((c0 + c) * p.Hkv + g) * p.part_bytes);
+      const float2 v = *reinterpret_cast<const float2*>(part + r * D + col);
+      const float f = fac[c * p.R + r];
+      x0 += f * v.x;
+      x1 += f * v.y;
+    }
+    const int t = r / p.G, hh = r % p.G;
+    uint16_t* dst = p.o + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + col;
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(x0 * inv[r], x1 * inv[r]);
+  }
+}
+
+int64_t max_items(int n_seqs, int Hkv, int window, int64_t max_ctx_len) {
+  int64_t cached = window > 0 ? (max_ctx_len < window ? max_ctx_len : window - 1) : max_ctx_len;
+  int64_t nsp = (cached + SPLIT - 1) / SPLIT;
+  if (nsp < 1) nsp = 1;
+  return (int64_t)n_seqs * Hkv * nsp;
+}
+
+template <int D, int MT>
+int launch_t(DecParams& p, int n_items_max, cudaStream_t stream) {
+  using SM = DecSmem<D, MT>;
+  static int sms = 0;
+  if (!sms) {
+    int dev;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  plan_kernel<<<1, 1024, 0, stream>>>(p);
+  cudaFuncSetAttribute(decode_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::BYTES);
+  int per_sm = 2;
+  int grid = sms * per_sm;
+  if (grid > n_items_max) grid = n_items_max;
+  if (grid < 1) grid = 1;
+  decode_kernel<D, MT><<<grid, DEC_THREADS, SM::BYTES, stream>>>(p);
+  {
+    const int64_t max_nsp = max_items(p.n_seqs, p.Hkv, p.window, p.max_ctx_len) / ((int64_t)p.n_seqs * p.Hkv);
+    if (max_nsp > 1) {
+      const size_t msm = ((size_t)max_nsp + 1) * p.R * sizeof(float);
+      if (msm > 48 * 1024)
+        cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msm);
+      merge_kernel<D><<<p.n_seqs * p.Hkv, 256, msm, stream>>>(p);
+    }
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("hybrid_decode_fwd: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int n_seqs, int n_qt, int Hq, int Hkv, int d, int window, int64_t max_ctx_len) {
+  const int G = Hq / Hkv;
+  const int rows = n_qt * G;
+  WsLayout L(n_seqs, rows, d, max_items(n_seqs, Hkv, window, max_ctx_len));
+  return L.bytes;
+}
+
+int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
+  const hswa_pool* pool = Lc.pool;
+  const hswa_pool_desc& D = pool->desc;
+  DecParams p{};
+  p.n_seqs = Lc.n_seqs;
+  p.n_qt = Lc.n_qt;
+  p.Hq = Lc.Hq;
+  p.Hkv = Lc.Hkv;
+  p.G = Lc.Hq / Lc.Hkv;
+  p.R = p.n_qt * p.G;
+  p.window = Lc.window;
+  p.q = Lc.q;
+  p.k_new = Lc.k_new;
+  p.v_new = Lc.v_new;
+  p.o = Lc.o;
+  p.ctx_len = Lc.ctx_len;
+  p.max_ctx_len = Lc.max_ctx_len;
+  p.seq_ids = Lc.seq_ids;
+  p.page_table = Lc.page_table;
+  p.pt_stride = Lc.pt_stride;
+  p.src_k = Lc.window > 0 ? pool->ring_k : pool->page_k;
+  p.src_v = Lc.window > 0 ? pool->ring_v : pool->page_v;
+  p.n_swa = D.n_swa_layers;
+  p.ring_layer = Lc.ring_layer;
+  p.max_seqs = D.max_seqs;
+  p.full_layer = Lc.full_layer;
+  p.pages = D.pages_per_full_layer;
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)Lc.d));
+  p.ws = static_cast<uint8_t*>(Lc.workspace);
+  p.err = pool->err;
+  const int64_t mi = max_items(p.n_seqs, p.Hkv, p.window, p.max_ctx_len);
+  WsLayout WL(p.n_seqs, p.R, Lc.d, mi);
+  p.part_off = WL.part_off;
+  p.part_bytes = WL.part_bytes_per_item;
+  if (p.R > 32) {
+    set_error("hybrid_decode_fwd: n_q_per_seq * (n_q_heads / n_kv_heads) = %d rows per KV head; at most 32 supported",
+              p.R);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  const int nmax = mi > 0x7fffffff ? 0x7fffffff : (int)mi;
+  if (Lc.d == 128) {
+    return p.R <= 16 ? launch_t<128, 1>(p, nmax, stream) : launch_t<128, 2>(p, nmax, stream);
+  }
+  return p.R <= 16 ? launch_t<64, 1>(p, nmax, stream) : launch_t<64, 2>(p, nmax, stream);
+}
+
+}  // namespace hswa

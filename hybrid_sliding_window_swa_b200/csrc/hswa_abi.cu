@@ -1,0 +1,439 @@
+// hswa_abi.cu -- the C ABI of libhswa.so: argument validation, dual-pool carving,
+// TMA descriptor encoding and dispatch to the kernels. No exception crosses the
+// boundary; every call returns a status and leaves a message in hswa_last_error().
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <new>
+
+#include "internal.h"
+
+namespace hswa {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_error("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) gs[i] = strides_bytes[i];
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return false;
+  }
+  return true;
+}
+
+static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int check_desc(const hswa_pool_desc* d) {
+  if (!d) {
+    set_error("null pool descriptor");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (d->n_swa_layers < 0 || d->n_full_layers < 0 || d->n_kv_heads < 1 || d->max_seqs < 0 ||
+      d->pages_per_full_layer < 0 || d->reserved != 0) {
+    set_error("invalid pool descriptor (negative count, zero KV heads or reserved != 0)");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (d->window < 1) {
+    set_error("window must be >= 1 (got %d)", d->window);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (d->head_dim != 64 && d->head_dim != 128) {
+    set_error("head_dim %d unsupported (64 or 128)", d->head_dim);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (d->page_size != 64) {
+    set_error("page_size %d unsupported (64)", d->page_size);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  return HSWA_OK;
+}
+
+static int check_heads(const hswa_pool* pool, int n_q_heads) {
+  const int hkv = pool->desc.n_kv_heads;
+  if (n_q_heads < 1 || n_q_heads % hkv != 0 || n_q_heads / hkv > 16 || n_q_heads > 65535) {
+    set_error("n_q_heads %d must be a positive multiple of n_kv_heads %d with ratio <= 16", n_q_heads, hkv);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  return HSWA_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace hswa
+
+using namespace hswa;
+
+extern "C" {
+
+const char* hswa_last_error(void) { return g_err; }
+
+int kv_pool_layout(const hswa_pool_desc* desc, size_t* bytes_total, size_t* bytes_swa, size_t* bytes_full) {
+  int rc = check_desc(desc);
+  if (rc) return rc;
+  const size_t e = 2;
+  const size_t swa = round256(2 * (size_t)desc->max_seqs * desc->n_swa_layers * desc->n_kv_heads *
+                              (size_t)desc->window * desc->head_dim * e);
+  const size_t full = round256(2 * (size_t)desc->n_full_layers * (size_t)desc->pages_per_full_layer *
+                               desc->n_kv_heads * (size_t)desc->page_size * desc->head_dim * e);
+  if (bytes_swa) *bytes_swa = swa;
+  if (bytes_full) *bytes_full = full;
+  if (bytes_total) *bytes_total = swa + full + 256;
+  return HSWA_OK;
+}
+
+int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa_pool** out) {
+  if (!out) {
+    set_error("kv_pool_create: null output handle");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  size_t total = 0, swa = 0, full = 0;
+  int rc = kv_pool_layout(desc, &total, &swa, &full);
+  if (rc) return rc;
+  if (!dev_mem || (reinterpret_cast<uintptr_t>(dev_mem) & 255u) != 0) {
+    set_error("kv_pool_create: device memory must be non-null and 256-byte aligned");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (bytes < total) {
+    set_error("kv_pool_create: %zu bytes given, layout needs %zu", bytes, total);
+    return HSWA_ERR_OUT_OF_MEMORY;
+  }
+  hswa_pool* p = new (std::nothrow) hswa_pool();
+  if (!p) {
+    set_error("kv_pool_create: host allocation failed");
+    return HSWA_ERR_OUT_OF_MEMORY;
+  }
+  p->desc = *desc;
+  cudaGetDevice(&p->device);
+  p->base = static_cast<uint8_t*>(dev_mem);
+  p->bytes_swa = swa;
+  p->bytes_full = full;
+  const size_t ring_half = (size_t)desc->max_seqs * desc->n_swa_layers * desc->n_kv_heads * (size_t)desc->window *
+                           desc->head_dim;
+  const size_t page_half = (size_t)desc->n_full_layers * (size_t)desc->pages_per_full_layer * desc->n_kv_heads *
+                           (size_t)desc->page_size * desc->head_dim;
+  p->ring_k = reinterpret_cast<uint16_t*>(p->base);
+  p->ring_v = p->ring_k + ring_half;
+  p->page_k = reinterpret_cast<uint16_t*>(p->base + swa);
+  p->page_v = p->page_k + page_half;
+  p->err = reinterpret_cast<int*>(p->base + swa + full);
+  const uint64_t D = desc->head_dim;
+  p->ring_tma = false;
+  const uint64_t ring_rows = (uint64_t)desc->max_seqs * desc->n_swa_layers * desc->n_kv_heads;
+  if (desc->window % 128 == 0 && ring_rows > 0) {
+    const uint64_t dims[3] = {D, (uint64_t)desc->window, ring_rows};
+    const uint64_t strides[2] = {D * 2, (uint64_t)desc->window * D * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!make_tmap_bf16(&p->tm_ring_k, p->ring_k, 3, dims, strides, box) ||
+        !make_tmap_bf16(&p->tm_ring_v, p->ring_v, 3, dims, strides, box)) {
+      delete p;
+      return HSWA_ERR_CUDA;
+    }
+    p->ring_tma = true;
+  }
+  p->page_tma = false;
+  const uint64_t page_rows = (uint64_t)desc->n_full_layers * desc->pages_per_full_layer * desc->n_kv_heads;
+  if (page_rows > 0) {
+    if (page_rows > 0x7FFFFFFFull) {
+      set_error("kv_pool_create: too many (layer, page, head) rows for 32-bit TMA coordinates");
+      delete p;
+      return HSWA_ERR_UNSUPPORTED_SHAPE;
+    }
+    const uint64_t dims[3] = {D, (uint64_t)desc->page_size, page_rows};
+    const uint64_t strides[2] = {D * 2, (uint64_t)desc->page_size * D * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if (!make_tmap_bf16(&p->tm_page_k, p->page_k, 3, dims, strides, box) ||
+        !make_tmap_bf16(&p->tm_page_v, p->page_v, 3, dims, strides, box)) {
+      delete p;
+      return HSWA_ERR_CUDA;
+    }
+    p->page_tma = true;
+  }
+  cudaError_t e = cudaMemset(p->err, 0, 256);
+  if (e != cudaSuccess) {
+    set_error("kv_pool_create: clearing the error word failed: %s", cudaGetErrorString(e));
+    delete p;
+    return HSWA_ERR_CUDA;
+  }
+  *out = p;
+  return HSWA_OK;
+}
+
+int kv_pool_destroy(hswa_pool* pool) {
+  delete pool;
+  return HSWA_OK;
+}
+
+int kv_pool_append(hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_ids, const int64_t* start_pos,
+                   int n_tok, const hswa_bf16* k, const hswa_bf16* v, const int32_t* page_table, int pt_stride,
+                   void* stream) {
+  if (!pool) {
+    set_error("kv_pool_append: null pool");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  if (layer < 0 || layer >= D.n_swa_layers + D.n_full_layers) {
+    set_error("kv_pool_append: layer %d out of range", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (n_seqs < 0 || n_tok < 0) {
+    set_error("kv_pool_append: negative sizes");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (n_seqs == 0 || n_tok == 0) return HSWA_OK;
+  const bool is_swa = layer < D.n_swa_layers;
+  if (!k || !v || !start_pos || !aligned16(k) || !aligned16(v) || (is_swa && !seq_ids) ||
+      (!is_swa && (!page_table || pt_stride < 1))) {
+    set_error("kv_pool_append: missing or misaligned device pointer");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  return launch_append(pool, layer, n_seqs, seq_ids, start_pos, n_tok, k, v, page_table, pt_stride,
+                       static_cast<cudaStream_t>(stream));
+}
+
+static int build_q_map(CUtensorMap* m, const void* base, int B, int n_q, int H, int d) {
+  const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)n_q, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)H * d * 2, (uint64_t)n_q * H * d * 2};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  return make_tmap_bf16(m, base, 4, dims, strides, box) ? HSWA_OK : HSWA_ERR_CUDA;
+}
+
+int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k, const hswa_bf16* v,
+                    hswa_bf16* o, int B, int n_q, const int64_t* start_pos, const int32_t* seq_ids, int n_q_heads,
+                    void* stream) {
+  if (!pool) {
+    set_error("swa_prefill_fwd: null pool");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  if (layer < 0 || layer >= D.n_swa_layers) {
+    set_error("swa_prefill_fwd: layer %d is not a sliding-window layer of this pool", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  int rc = check_heads(pool, n_q_heads);
+  if (rc) return rc;
+  if (B < 0 || n_q < 0 || B > 65535) {
+    set_error("swa_prefill_fwd: bad B or n_q");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (B == 0 || n_q == 0) return HSWA_OK;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) {
+    set_error("swa_prefill_fwd: missing or misaligned tensor pointer");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (start_pos && !seq_ids) {
+    set_error("swa_prefill_fwd: seq_ids are required with start_pos");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  PrefillLaunch L{};
+  L.B = B;
+  L.n_q = n_q;
+  L.Hq = n_q_heads;
+  L.Hkv = D.n_kv_heads;
+  L.d = D.head_dim;
+  L.window = D.window;
+  L.start_pos = start_pos;
+  L.seq_ids = seq_ids;
+  L.o = o;
+  L.pool = pool;
+  L.ring_layer = layer;
+  if ((rc = build_q_map(&L.tm_q, q, B, n_q, n_q_heads, D.head_dim))) return rc;
+  if ((rc = build_q_map(&L.tm_k, k, B, n_q, D.n_kv_heads, D.head_dim))) return rc;
+  if ((rc = build_q_map(&L.tm_v, v, B, n_q, D.n_kv_heads, D.head_dim))) return rc;
+  return launch_prefill(L, static_cast<cudaStream_t>(stream));
+}
+
+int full_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, hswa_bf16* o, int B, int n_q,
+                     const int64_t* start_pos, const int32_t* page_table, int pt_stride, int n_q_heads,
+                     void* stream) {
+  if (!pool) {
+    set_error("full_prefill_fwd: null pool");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  if (layer < D.n_swa_layers || layer >= D.n_swa_layers + D.n_full_layers) {
+    set_error("full_prefill_fwd: layer %d is not a full layer of this pool", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  int rc = check_heads(pool, n_q_heads);
+  if (rc) return rc;
+  if (B < 0 || n_q < 0 || B > 65535) {
+    set_error("full_prefill_fwd: bad B or n_q");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (B == 0 || n_q == 0) return HSWA_OK;
+  if (!q || !o || !aligned16(q) || !aligned16(o) || !page_table || pt_stride < 1 || !pool->page_tma) {
+    set_error("full_prefill_fwd: missing tensor pointer, page table, or pool pages");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  PrefillLaunch L{};
+  L.B = B;
+  L.n_q = n_q;
+  L.Hq = n_q_heads;
+  L.Hkv = D.n_kv_heads;
+  L.d = D.head_dim;
+  L.window = 0;
+  L.start_pos = start_pos;
+  L.page_table = page_table;
+  L.pt_stride = pt_stride;
+  L.o = o;
+  L.pool = pool;
+  L.full_layer = layer - D.n_swa_layers;
+  if ((rc = build_q_map(&L.tm_q, q, B, n_q, n_q_heads, D.head_dim))) return rc;
+  L.tm_k = pool->tm_page_k;
+  L.tm_v = pool->tm_page_v;
+  return launch_prefill(L, static_cast<cudaStream_t>(stream));
+}
+
+int hybrid_decode_workspace_size(const hswa_pool* pool, int n_seqs, int n_q_per_seq, int n_q_heads,
+                                 int64_t max_ctx_len, size_t* bytes) {
+  if (!pool || !bytes || n_seqs < 0 || n_q_per_seq < 1 || n_q_per_seq > 8 || max_ctx_len < 0) {
+    set_error("hybrid_decode_workspace_size: bad arguments");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  int rc = check_heads(pool, n_q_heads);
+  if (rc) return rc;
+  const hswa_pool_desc& D = pool->desc;
+  // sized for a full layer, the larger of the two layer kinds
+  *bytes = decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, D.n_kv_heads, D.head_dim, 0, max_ctx_len);
+  return HSWA_OK;
+}
+
+int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
+                      const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq, const int64_t* ctx_len,
+                      int64_t max_ctx_len, const int32_t* seq_ids, const int32_t* page_table, int pt_stride,
+                      int n_q_heads, void* workspace, size_t ws_bytes, void* stream) {
+  if (!pool) {
+    set_error("hybrid_decode_fwd: null pool");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  if (layer < 0 || layer >= D.n_swa_layers + D.n_full_layers) {
+    set_error("hybrid_decode_fwd: layer %d out of range", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  int rc = check_heads(pool, n_q_heads);
+  if (rc) return rc;
+  if (n_seqs < 0 || n_q_per_seq < 1 || n_q_per_seq > 8 || max_ctx_len < 0) {
+    set_error("hybrid_decode_fwd: bad sizes (n_q_per_seq must be 1..8)");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (n_seqs == 0) return HSWA_OK;
+  const bool is_swa = layer < D.n_swa_layers;
+  if (!q || !k_new || !v_new || !o || !ctx_len || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned16(o) || (is_swa && !seq_ids) || (!is_swa && (!page_table || pt_stride < 1))) {
+    set_error("hybrid_decode_fwd: missing or misaligned device pointer");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const size_t need = decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, D.n_kv_heads, D.head_dim,
+                                             is_swa ? D.window : 0, max_ctx_len);
+  if (ws_bytes < need || (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)))) {
+    set_error("hybrid_decode_fwd: workspace of %zu bytes (256-aligned) needed, %zu given", need, ws_bytes);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  DecodeLaunch L{};
+  L.n_seqs = n_seqs;
+  L.n_qt = n_q_per_seq;
+  L.Hq = n_q_heads;
+  L.Hkv = D.n_kv_heads;
+  L.d = D.head_dim;
+  L.window = is_swa ? D.window : 0;
+  L.q = q;
+  L.k_new = k_new;
+  L.v_new = v_new;
+  L.o = o;
+  L.ctx_len = ctx_len;
+  L.max_ctx_len = max_ctx_len;
+  L.seq_ids = seq_ids;
+  L.page_table = page_table;
+  L.pt_stride = pt_stride;
+  L.pool = pool;
+  L.ring_layer = is_swa ? layer : 0;
+  L.full_layer = is_swa ? 0 : layer - D.n_swa_layers;
+  L.workspace = workspace;
+  L.ws_bytes = ws_bytes;
+  return launch_decode(L, static_cast<cudaStream_t>(stream));
+}
+
+int window_safe_len(const int64_t* match_len, const int64_t* cached_len, const uint32_t* slot_valid, int32_t W,
+                    int32_t n_req, int64_t* out_len, void* stream) {
+  if (W < 1 || n_req < 0) {
+    set_error("window_safe_len: W must be >= 1 and n_req >= 0");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (n_req == 0) return HSWA_OK;
+  if (!match_len || !cached_len || !slot_valid || !out_len) {
+    set_error("window_safe_len: null device pointer");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  return launch_window_safe_len(match_len, cached_len, slot_valid, W, n_req, out_len,
+                                static_cast<cudaStream_t>(stream));
+}
+
+int hswa_pool_check_error(hswa_pool* pool, int* device_code) {
+  if (!pool || !device_code) {
+    set_error("hswa_pool_check_error: null argument");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    set_error("hswa_pool_check_error: device synchronisation failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  int code = 0;
+  e = cudaMemcpy(&code, pool->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(pool->err, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    set_error("hswa_pool_check_error: reading the error word failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  *device_code = code;
+  return HSWA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,83 @@
+// internal.h -- host-side pool object and kernel launch interfaces of libhswa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hswa.h"
+
+struct hswa_pool {
+  hswa_pool_desc desc;
+  int device;
+  uint8_t* base;
+  size_t bytes_swa, bytes_full;
+  uint16_t* ring_k;  // [max_seqs][n_swa][Hkv][W][d]
+  uint16_t* ring_v;
+  uint16_t* page_k;  // [n_full][pages][Hkv][page_size][d]
+  uint16_t* page_v;
+  int* err;          // device error word
+  bool ring_tma;     // W is a multiple of 128: ring tiles can be fetched with one TMA box
+  CUtensorMap tm_ring_k, tm_ring_v;
+  bool page_tma;
+  CUtensorMap tm_page_k, tm_page_v;
+};
+
+namespace hswa {
+
+// Thread-local error message of the ABI layer.
+void set_error(const char* fmt, ...);
+
+// Encode a 2-5 dimensional bf16 tiled tensor map with 128-byte swizzle.
+// dims/strides: innermost first; strides in bytes for dims 1.. (dim 0 is contiguous).
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box);
+
+int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_ids,
+                  const int64_t* start_pos, int n_tok, const uint16_t* k, const uint16_t* v,
+                  const int32_t* page_table, int pt_stride, cudaStream_t stream);
+
+int launch_window_safe_len(const int64_t* m, const int64_t* c, const uint32_t* valid, int W, int n_req,
+                           int64_t* out, cudaStream_t stream);
+
+struct PrefillLaunch {
+  // problem
+  int B, n_q, Hq, Hkv, d;
+  int window;  // >= 1 for SWA, 0 for full causal
+  const int64_t* start_pos;  // device, may be null (all zero)
+  const int32_t* seq_ids;    // SWA ring rows
+  const int32_t* page_table; // full layers
+  int pt_stride;
+  uint16_t* o;
+  // pool
+  const hswa_pool* pool;
+  int ring_layer;      // SWA layer index within the ring (SWA)
+  int full_layer;      // full layer index within the paged pool (full)
+  // tensor maps built by the ABI layer
+  CUtensorMap tm_q, tm_k, tm_v;  // tm_k/tm_v: chunk K/V (SWA) or pages (full)
+};
+
+int launch_prefill(const PrefillLaunch& L, cudaStream_t stream);
+
+struct DecodeLaunch {
+  int n_seqs, n_qt, Hq, Hkv, d;
+  int window;  // >= 1 SWA (ring), 0 full (pages)
+  const uint16_t* q;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* o;
+  const int64_t* ctx_len;
+  int64_t max_ctx_len;
+  const int32_t* seq_ids;
+  const int32_t* page_table;
+  int pt_stride;
+  const hswa_pool* pool;
+  int ring_layer, full_layer;
+  void* workspace;
+  size_t ws_bytes;
+};
+
+size_t decode_workspace_bytes(int n_seqs, int n_qt, int Hq, int Hkv, int d, int window, int64_t max_ctx_len);
+int launch_decode(const DecodeLaunch& L, cudaStream_t stream);
+
+}  // namespace hswa

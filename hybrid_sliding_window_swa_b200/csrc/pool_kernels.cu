@@ -1,0 +1,149 @@
+// pool_kernels.cu -- KV commit into the dual pool and the window-safe prefix-match length.
+//
+// Rolling buffer: position t lives in slot t mod W ("Sliding Window Attention (SWA)
+// no riron to jisso", section "Rolling Buffer KV Cache", eq. (7)). Paged pool: position
+// t of a sequence lives in page page_table[t / page_size], row t mod page_size.
+// Window-safe length: "MiMo v2.5 inference optimisation", section "KV cache redesign".
+#include "common.cuh"
+#include "internal.h"
+
+namespace hswa {
+
+// One thread moves 16 bytes (8 bf16). Rows are (sequence b, token t, KV head g) of d elements.
+template <int D>
+__global__ void __launch_bounds__(256) append_kernel(
+    const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int n_seqs, int n_tok, int Hkv,
+    const int64_t* __restrict__ start_pos, const int32_t* __restrict__ seq_ids,
+    const int32_t* __restrict__ page_table, int pt_stride,
+    uint16_t* __restrict__ dst_k, uint16_t* __restrict__ dst_v, int is_swa, int W, int n_swa, int layer,
+    int max_seqs, int64_t pages, int page_size, int* err) {
+  constexpr int VEC = 8;
+  constexpr int PER_ROW = D / VEC;
+  const int64_t rows = (int64_t)n_seqs * n_tok * Hkv;
+  const int64_t total = rows * PER_ROW;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = idx / PER_ROW;
+    const int c = (int)(idx % PER_ROW);
+    const int g = (int)(row % Hkv);
+    const int64_t bt = row / Hkv;
+    const int t = (int)(bt % n_tok);
+    const int b = (int)(bt / n_tok);
+    const int64_t pos = start_pos[b] + t;
+    int64_t dst_row;
+    if (is_swa) {
+      if (t < n_tok - W) continue;  // overwritten later in the same chunk
+      const int seq = seq_ids[b];
+      if (seq < 0 || seq >= max_seqs || pos < 0) {
+        record_error(err, HSWA_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      dst_row = (((int64_t)seq * n_swa + layer) * Hkv + g) * W + (pos % W);
+    } else {
+      const int64_t lp = pos / page_size;
+      if (pos < 0 || lp >= pt_stride) {
+        record_error(err, HSWA_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      const int32_t page = page_table[(int64_t)b * pt_stride + lp];
+      if (page < 0 || page >= pages) {
+        record_error(err, HSWA_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      dst_row = (((int64_t)layer * pages + page) * Hkv + g) * page_size + (pos % page_size);
+    }
+    const uint4* src_k = reinterpret_cast<const uint4*>(k + row * D) + c;
+    const uint4* src_v = reinterpret_cast<const uint4*>(v + row * D) + c;
+    uint4* out_k = reinterpret_cast<uint4*>(dst_k + dst_row * D) + c;
+    uint4* out_v = reinterpret_cast<uint4*>(dst_v + dst_row * D) + c;
+    *out_k = __ldg(src_k);
+    *out_v = __ldg(src_v);
+  }
+}
+
+int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_ids,
+                  const int64_t* start_pos, int n_tok, const uint16_t* k, const uint16_t* v,
+                  const int32_t* page_table, int pt_stride, cudaStream_t stream) {
+  const hswa_pool_desc& D = pool->desc;
+  const bool is_swa = layer < D.n_swa_layers;
+  const int64_t total = (int64_t)n_seqs * n_tok * D.n_kv_heads * (D.head_dim / 8);
+  if (total == 0) return HSWA_OK;
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, pool->device);
+  const int64_t want = (total + 255) / 256;
+  const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+  uint16_t* dk = is_swa ? pool->ring_k : pool->page_k;
+  uint16_t* dv = is_swa ? pool->ring_v : pool->page_v;
+  const int l = is_swa ? layer : layer - D.n_swa_layers;
+  if (D.head_dim == 128)
+    append_kernel<128><<<grid, 256, 0, stream>>>(k, v, n_seqs, n_tok, D.n_kv_heads, start_pos, seq_ids,
+                                                  page_table, pt_stride, dk, dv, is_swa, D.window,
+                                                  D.n_swa_layers, l, D.max_seqs, D.pages_per_full_layer,
+                                                  D.page_size, pool->err);
+  else
+    append_kernel<64><<<grid, 256, 0, stream>>>(k, v, n_seqs, n_tok, D.n_kv_heads, start_pos, seq_ids,
+                                                 page_table, pt_stride, dk, dv, is_swa, D.window,
+                                                 D.n_swa_layers, l, D.max_seqs, D.pages_per_full_layer,
+                                                 D.page_size, pool->err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("kv_pool_append: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
+// One thread per request. With the ring holding positions [max(0, C-W), C):
+//  * C > W: the only resumable lengths are 0 and C (every other tail reaches a
+//    position older than C - W); C needs m >= C and all W slots valid.
+//  * C <= W: slot s holds position s; L is safe iff L <= C and slots 0..L-1 are
+//    valid, so the answer is min(m, C, first invalid slot).
+__global__ void __launch_bounds__(128) window_safe_len_kernel(const int64_t* __restrict__ m,
+                                                              const int64_t* __restrict__ c,
+                                                              const uint32_t* __restrict__ valid, int W,
+                                                              int n_req, int64_t* __restrict__ out) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= n_req) return;
+  const int words = (W + 31) >> 5;
+  const uint32_t* vr = valid + (int64_t)r * words;
+  const int64_t M = m[r], C = c[r];
+  int64_t res;
+  if (M < 0 || C < 0) {
+    res = 0;
+  } else if (C > W) {
+    bool all = true;
+    for (int w = 0; w < words && all; ++w) {
+      const int bits = (w == words - 1) ? (W - 32 * w) : 32;
+      const uint32_t need = bits == 32 ? 0xFFFFFFFFu : ((1u << bits) - 1u);
+      all = (__ldg(vr + w) & need) == need;
+    }
+    res = (all && M >= C) ? C : 0;
+  } else {
+    // first invalid slot among 0 .. C-1 (C <= W)
+    int64_t first_bad = C;
+    for (int w = 0; w * 32 < C; ++w) {
+      const uint32_t inv = ~__ldg(vr + w);
+      if (inv) {
+        const int64_t s = 32 * (int64_t)w + (__ffs(inv) - 1);
+        if (s < first_bad) first_bad = s;
+        break;
+      }
+    }
+    res = M < first_bad ? M : first_bad;
+  }
+  out[r] = res;
+}
+
+int launch_window_safe_len(const int64_t* m, const int64_t* c, const uint32_t* valid, int W, int n_req,
+                           int64_t* out, cudaStream_t stream) {
+  if (n_req == 0) return HSWA_OK;
+  window_safe_len_kernel<<<(n_req + 127) / 128, 128, 0, stream>>>(m, c, valid, W, n_req, out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("window_safe_len: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
+}  // namespace hswa

@@ -1,0 +1,193 @@
+/*
+ * hswa.h -- hybrid sliding-window attention on NVIDIA B200 (sm_100a): C ABI of libhswa.so.
+ *
+ * What it computes. For a query at absolute position i the sliding-window layers
+ * attend the keys j with max(0, i - W + 1) <= j <= i and the full layers attend
+ * 0 <= j <= i, with softmax(q.k / sqrt(head_dim)) weights on the values
+ * ("Sliding Window Attention (SWA) no riron to jisso", disassemble-channel.com,
+ * section "formal definition", eqs. (1)-(5)). Several query heads share one KV
+ * head: query head h reads KV head h / (n_q_heads / n_kv_heads) (same page,
+ * section "Mistral: SWA and GQA"). Keys and values of the SWA layers live in a
+ * rolling buffer of W slots with slot = position mod W (same page, section
+ * "Rolling Buffer KV Cache", eq. (7)); keys and values of the full layers live
+ * in a paged pool sized by the sequence length. The two pools together are the
+ * dual-pool KV cache of "MiMo v2.5 inference optimisation" (youngju.dev,
+ * section "KV cache redesign"), which also defines the window-safe prefix-match
+ * length.
+ *
+ * Conventions for every call.
+ *  - Returns HSWA_OK (0) or a negative HSWA_ERR_* code; hswa_last_error()
+ *    returns a message for the last failure on the calling thread.
+ *    No C++ exception crosses this boundary.
+ *  - Tensor arguments are raw device pointers owned by the caller (normally
+ *    torch tensors), contiguous in the layouts stated below, 16-byte aligned.
+ *    bf16 data is passed as its 16-bit pattern (hswa_bf16).
+ *  - Compute calls enqueue work on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and return without synchronising. Argument errors
+ *    found on the host return before anything is enqueued. Errors found on the
+ *    device (a page id out of range, a context length above the declared
+ *    maximum, a wait that ran out) are recorded in the pool's device error word
+ *    and read back with hswa_pool_check_error().
+ *  - The library never allocates device memory. Pool memory and the decode
+ *    workspace are passed in by the caller.
+ *  - Supported shapes: head_dim 64 or 128, n_q_heads a multiple of n_kv_heads,
+ *    n_q_heads / n_kv_heads <= 16, W >= 1, page_size 64. Anything else returns
+ *    HSWA_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef HSWA_H
+#define HSWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HSWA_API __attribute__((visibility("default")))
+#else
+#define HSWA_API
+#endif
+
+#define HSWA_OK 0
+#define HSWA_ERR_INVALID_ARG (-1)
+#define HSWA_ERR_UNSUPPORTED_SHAPE (-2)
+#define HSWA_ERR_OUT_OF_MEMORY (-3)
+#define HSWA_ERR_CUDA (-4)
+#define HSWA_ERR_TIMEOUT (-5)
+#define HSWA_ERR_DEVICE_BOUNDS (-6)
+
+typedef uint16_t hswa_bf16;
+typedef struct hswa_pool hswa_pool;
+
+/* Shape of a dual-pool KV cache.
+ * Layers 0 .. n_swa_layers-1 of the pool are sliding-window layers with a
+ * W-slot ring per (sequence, layer, KV head); layers n_swa_layers ..
+ * n_swa_layers+n_full_layers-1 are full layers whose token-slots are pages of
+ * page_size tokens, pages_per_full_layer pages per layer, shared by all
+ * sequences through a page table. */
+typedef struct hswa_pool_desc {
+  int32_t n_swa_layers;          /* >= 0 */
+  int32_t n_full_layers;         /* >= 0 */
+  int32_t window;                /* W >= 1 */
+  int32_t n_kv_heads;            /* >= 1 */
+  int32_t head_dim;              /* 64 or 128 */
+  int32_t page_size;             /* 64 */
+  int32_t max_seqs;              /* number of ring rows (sequence ids 0 .. max_seqs-1) */
+  int32_t reserved;              /* must be 0 */
+  int64_t pages_per_full_layer;  /* >= 0 */
+} hswa_pool_desc;
+
+/* Dual-pool sizing ("MiMo v2.5 inference optimisation", section "KV cache redesign":
+ * the SWA pool holds W tokens, O(W); the full pool is sized by length, O(N)).
+ * Device memory layout, from the base pointer:
+ *   ring  K then V : [2][max_seqs][n_swa_layers][n_kv_heads][W][head_dim] bf16
+ *   pages K then V : [2][n_full_layers][pages_per_full_layer][n_kv_heads][page_size][head_dim] bf16
+ *   error word     : 256 bytes (int32 device error code + spare)
+ * each region starting on a 256-byte boundary.
+ * bytes_swa  = 2 * max_seqs * n_swa_layers * n_kv_heads * W * head_dim * 2, rounded up to 256;
+ * bytes_full = 2 * n_full_layers * pages * n_kv_heads * page_size * head_dim * 2, rounded up to 256;
+ * bytes_total = bytes_swa + bytes_full + 256.  Any output pointer may be NULL. */
+HSWA_API int kv_pool_layout(const hswa_pool_desc* desc, size_t* bytes_total, size_t* bytes_swa,
+                   size_t* bytes_full);
+
+/* Carve a pool out of caller-owned device memory `dev_mem` of `bytes` bytes
+ * (>= bytes_total, 256-byte aligned) on the current CUDA device. The library
+ * keeps views and TMA descriptors only; it does not initialise the K/V slots,
+ * and clears the error word. The caller frees dev_mem after kv_pool_destroy(). */
+HSWA_API int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa_pool** out);
+
+/* Release the host-side handle (not the device memory). NULL is accepted. */
+HSWA_API int kv_pool_destroy(hswa_pool* pool);
+
+/* Commit n_tok new tokens per sequence into layer `layer`.
+ *  k, v       [n_seqs][n_tok][n_kv_heads][head_dim] bf16, token t of row b sits at
+ *             absolute position start_pos[b] + t.
+ *  start_pos  device int64[n_seqs], >= 0.
+ *  seq_ids    device int32[n_seqs], ring row of each sequence (SWA layers; may be NULL for full layers).
+ *  page_table device int32[n_seqs][pt_stride]: row b lists the physical page of logical page
+ *             p = position / page_size of sequence b (full layers; may be NULL for SWA layers).
+ * SWA layer: only the last min(n_tok, W) tokens are written, each to slot position mod W
+ * ("Rolling Buffer KV Cache", eq. (7)); earlier tokens of the chunk would be
+ * overwritten within the same chunk. Full layer: every token goes to
+ * page_table[b][pos / page_size], row pos mod page_size. A page id outside
+ * [0, pages_per_full_layer) or a logical page >= pt_stride is skipped and
+ * recorded as HSWA_ERR_DEVICE_BOUNDS. */
+HSWA_API int kv_pool_append(hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_ids,
+                   const int64_t* start_pos, int n_tok, const hswa_bf16* k, const hswa_bf16* v,
+                   const int32_t* page_table, int pt_stride, void* stream);
+
+/* Causal sliding-window attention for one chunk of n_q new tokens per sequence
+ * ("formal definition", eqs. (1)-(5), window W of the pool), on tensor cores.
+ *  q, o    [B][n_q][n_q_heads][head_dim] bf16 (o written, rows in the chunk only)
+ *  k, v    [B][n_q][n_kv_heads][head_dim] bf16, the chunk's own keys and values
+ *  start_pos device int64[B] = absolute position of the chunk's first token, or NULL for 0.
+ *  seq_ids   device int32[B] ring rows (needed when start_pos is not NULL).
+ * Keys before start_pos[b] are read from the ring of layer `layer` (an SWA layer),
+ * which must hold positions [start_pos[b] - W, start_pos[b]) as committed by
+ * kv_pool_append: attention reads the ring as it was before this chunk; commit
+ * the chunk with kv_pool_append afterwards. Key tiles wholly outside every
+ * query's window are skipped, not masked. fp32 accumulation and softmax. */
+HSWA_API int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k,
+                    const hswa_bf16* v, hswa_bf16* o, int B, int n_q, const int64_t* start_pos,
+                    const int32_t* seq_ids, int n_q_heads, void* stream);
+
+/* Full causal attention for one chunk of n_q tokens per sequence over the paged
+ * pool of full layer `layer`: query i = start_pos[b] + t attends positions 0..i,
+ * all read through the page table (the chunk itself must already be appended).
+ *  q, o      [B][n_q][n_q_heads][head_dim] bf16
+ *  start_pos device int64[B] (NULL for 0); page_table device int32[B][pt_stride]. */
+HSWA_API int full_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, hswa_bf16* o, int B,
+                     int n_q, const int64_t* start_pos, const int32_t* page_table, int pt_stride,
+                     int n_q_heads, void* stream);
+
+/* Bytes of device workspace hybrid_decode_fwd needs for these arguments. */
+HSWA_API int hybrid_decode_workspace_size(const hswa_pool* pool, int n_seqs, int n_q_per_seq,
+                                 int n_q_heads, int64_t max_ctx_len, size_t* bytes);
+
+/* One decode step: n_q_per_seq (1..8; 4 = one token + three multi-token-prediction
+ * drafts) new query tokens per sequence at positions L .. L+n_q_per_seq-1, where
+ * L = ctx_len[b] cached tokens. Draft t attends the cached keys in its window
+ * plus new tokens 0..t (causal among themselves). SWA layer: the cached keys
+ * come from the ring, which must hold positions [L - W, L); full layer: from the
+ * page table, positions [0, L). The new keys/values are read from k_new/v_new,
+ * not from the pool: commit them with kv_pool_append after acceptance.
+ * Split-KV: the cached keys are cut into splits that run in parallel and are
+ * merged with their log-sum-exp partials.
+ *  q, o          [n_seqs][n_q_per_seq][n_q_heads][head_dim] bf16
+ *  k_new, v_new  [n_seqs][n_q_per_seq][n_kv_heads][head_dim] bf16
+ *  ctx_len       device int64[n_seqs], 0 <= L <= max_ctx_len (else HSWA_ERR_DEVICE_BOUNDS)
+ *  seq_ids       device int32[n_seqs] ring rows (SWA layer)
+ *  page_table    device int32[n_seqs][pt_stride] (full layer)
+ *  workspace     device scratch of ws_bytes >= hybrid_decode_workspace_size(); its contents
+ *                on entry do not matter; calls sharing one workspace must not overlap. */
+HSWA_API int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
+                      const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq,
+                      const int64_t* ctx_len, int64_t max_ctx_len, const int32_t* seq_ids,
+                      const int32_t* page_table, int pt_stride, int n_q_heads, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* Window-safe prefix-match length ("MiMo v2.5 inference optimisation", section
+ * "KV cache redesign": a prefix-cache match may be reused only as far as the
+ * last W tokens before the resume point still have valid SWA slots).
+ * For request r with match length m = match_len[r] and cached length C = cached_len[r],
+ * whose ring holds positions [max(0, C-W), C) with slot s valid iff bit s%32 of
+ * slot_valid[r * ((W+31)/32) + s/32] is set:
+ *   out_len[r] = max { L in [0, m] : every position in [max(0, L-W), L) is held in a valid slot }.
+ * All arrays are device memory; results are exact integers. */
+HSWA_API int window_safe_len(const int64_t* match_len, const int64_t* cached_len,
+                    const uint32_t* slot_valid, int32_t W, int32_t n_req, int64_t* out_len,
+                    void* stream);
+
+/* Synchronise the device, return the pool's device error word in *device_code
+ * (0 if none, else a negative HSWA_ERR_* code) and clear it. */
+HSWA_API int hswa_pool_check_error(hswa_pool* pool, int* device_code);
+
+/* Message for the last failed call on this thread ("" if none). */
+HSWA_API const char* hswa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSWA_H */
