@@ -151,6 +151,12 @@ class KVPool:
         return ring, pages
 
     @property
+    def data(self) -> torch.Tensor:
+        """uint8 view of the K/V regions only (the library's error word that follows them excluded)."""
+        _, swa, full = kv_pool_layout(self.desc)
+        return self.memory[: swa + full]
+
+    @property
     def ring(self) -> torch.Tensor:
         """[2 (K,V)][max_seqs][n_swa_layers][Hkv][W][d] view of the rolling buffers."""
         return self._views()[0]

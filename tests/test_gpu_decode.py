@@ -20,7 +20,7 @@ def run_decode_case(seed, lens, n_qt, hq, hkv, d, W, kind, layer_swa=0, n_swa=1,
     desc = hs.PoolDesc(n_swa_layers=n_swa, n_full_layers=n_full, window=W, n_kv_heads=hkv, head_dim=d,
                        max_seqs=n + 2, pages_per_full_layer=total_pages)
     pool = hs.kv_pool_create(desc)
-    pool.memory.fill_(0xFF)
+    pool.data.fill_(0xFF)
     layer = layer_swa if kind == "swa" else n_swa
     seq_ids = (torch.arange(n, dtype=torch.int32) * 7 % (n + 2)).contiguous()
     pt = page_table_for(seed, n, pages_per_seq, total_pages).cuda() if kind == "full" else None
@@ -90,7 +90,7 @@ def test_ctx_len_above_declared_max_is_reported():
     desc = hs.PoolDesc(n_swa_layers=0, n_full_layers=1, window=128, n_kv_heads=1, head_dim=64, max_seqs=1,
                        pages_per_full_layer=4)
     pool = hs.kv_pool_create(desc)
-    pool.memory.zero_()
+    pool.data.zero_()
     q = torch.zeros(1, 1, 1, 64, dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(hs.hybrid_decode_workspace_size(pool, 1, 1, 1, 100), dtype=torch.uint8, device="cuda")
     pt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")

@@ -72,7 +72,7 @@ def test_ring_append_places_slot_pos_mod_w(w, hkv, d):
     desc = hs.PoolDesc(n_swa_layers=2, n_full_layers=0, window=w, n_kv_heads=hkv, head_dim=d, max_seqs=4,
                        pages_per_full_layer=0)
     pool = hs.kv_pool_create(desc)
-    pool.memory.zero_()
+    pool.data.zero_()
     seq_ids = torch.tensor([2, 0, 3], dtype=torch.int32)
     # append in several calls of different lengths: positions 0..T-1 per sequence
     T = 3 * w + 5
@@ -104,7 +104,7 @@ def test_page_append_follows_page_table():
     desc = hs.PoolDesc(n_swa_layers=1, n_full_layers=2, window=128, n_kv_heads=hkv, head_dim=d, max_seqs=1,
                        pages_per_full_layer=40)
     pool = hs.kv_pool_create(desc)
-    pool.memory.zero_()
+    pool.data.zero_()
     n_seqs, n_tok = 2, 300  # 5 pages each, last one partial
     pt = page_table_for(seed, n_seqs, 8, 40)
     layer = 2  # second full layer
@@ -128,7 +128,7 @@ def test_bad_page_id_is_recorded_not_written():
     desc = hs.PoolDesc(n_swa_layers=0, n_full_layers=1, window=1, n_kv_heads=1, head_dim=64, max_seqs=0,
                        pages_per_full_layer=4)
     pool = hs.kv_pool_create(desc)
-    pool.memory.zero_()
+    pool.data.zero_()
     k = torch.ones(1, 64, 1, 64, dtype=torch.bfloat16, device="cuda")
     pt = torch.tensor([[7]], dtype=torch.int32, device="cuda")  # page 7 does not exist
     hs.kv_pool_append(pool, 0, k, k, torch.zeros(1, dtype=torch.int64, device="cuda"), page_table=pt)

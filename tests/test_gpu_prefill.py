@@ -20,7 +20,7 @@ def run_swa_case(seed, B, n_q, W, hq, hkv, d, starts, sigma=1.0, layer=0, rows=N
     desc = hs.PoolDesc(n_swa_layers=layer + 1, n_full_layers=0, window=W, n_kv_heads=hkv, head_dim=d,
                        max_seqs=B + 1, pages_per_full_layer=0)
     pool = hs.kv_pool_create(desc)
-    pool.memory.fill_(0xFF)  # NaN bit patterns everywhere the kernel must not read
+    pool.data.fill_(0xFF)  # NaN bit patterns everywhere the kernel must not read
     seq_ids = torch.arange(B, dtype=torch.int32).flip(0) + 1  # ring rows 1..B, reversed
     qs, ks, vs = [], [], []
     for b in range(B):
@@ -108,7 +108,7 @@ def run_full_case(seed, B, n_q, hq, hkv, d, starts, layer=0, total_pages=None, r
     desc = hs.PoolDesc(n_swa_layers=0, n_full_layers=layer + 1, window=1, n_kv_heads=hkv, head_dim=d,
                        max_seqs=0, pages_per_full_layer=total_pages)
     pool = hs.kv_pool_create(desc)
-    pool.memory.fill_(0xFF)
+    pool.data.fill_(0xFF)
     pt = page_table_for(seed, B, max_pages, total_pages).cuda()
     qs = []
     for b in range(B):
