@@ -1,0 +1,601 @@
+"""Benchmark of the hybrid sliding-window attention hot path on B200.
+
+Default workload (one JSON line): Mistral-shaped sliding-window prefill of one 16K-token
+chunk, B=2, N=16384, W=4096, Hq=32, Hkv=8, head_dim=128, bf16 Q/K/V ~ N(0,1)/sqrt(2) from
+the seeded generator. One step = swa_prefill_fwd (band attention on tensor cores) +
+kv_pool_append (commit of the chunk's last W tokens into the rolling buffer). Useful
+FLOPs count only the (query, key) pairs inside the band: 4 * d * pairs * Hq * B.
+
+Secondary results in the same line (unless --no-secondary): the 512-token single-layer
+cases (W = 128, 512, 1), the hybrid 16K chunk after a 131072-token prefix (one SWA layer
+W=128 and one paged full layer), and the hybrid decode batch (256 sequences, log-uniform
+context lengths in [1K, 256K], 4 query tokens each, 6 SWA layers + 1 full layer) with
+window_safe_len over 4096 requests.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no data-path
+collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+import synth
+
+METRIC = "SWA/full prefill TFLOP/s (% BF16 peak); hybrid decode KV GB/s (% HBM peak)"
+SEED = 20261202
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------ workloads
+
+def gen(tag, layer, seq, pos0, n, h, d, sigma, device):
+    return synth.normal_bf16_rows(SEED, synth.stream_id(tag, layer, seq), pos0, n, h * d, sigma, device).view(n, h, d)
+
+
+class SwaPrefill16k:
+    """Mistral-shaped SWA prefill of one 16K chunk (B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128)."""
+    name = "swa_prefill_16k_B2_W4096_Hq32_Hkv8_d128"
+
+    def __init__(self, hs, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128, seq_offset=0):
+        self.hs = hs
+        self.B, self.N, self.W, self.Hq, self.Hkv, self.d = B, N, W, Hq, Hkv, d
+        self.sigma = 2 ** -0.5
+        self.seq_offset = seq_offset
+        dev = "cuda"
+        self.q = torch.stack([gen(synth.TAG_Q, 0, seq_offset + b, 0, N, Hq, d, self.sigma, dev) for b in range(B)])
+        self.k = torch.stack([gen(synth.TAG_K, 0, seq_offset + b, 0, N, Hkv, d, self.sigma, dev) for b in range(B)])
+        self.v = torch.stack([gen(synth.TAG_V, 0, seq_offset + b, 0, N, Hkv, d, self.sigma, dev) for b in range(B)])
+        self.o = torch.empty_like(self.q)
+        self.pool = hs.kv_pool_create(hs.PoolDesc(1, 0, W, Hkv, d, B, 0))
+        self.start = torch.zeros(B, dtype=torch.int64, device=dev)
+        self.seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
+        pairs = W * (W + 1) // 2 + (N - W) * W if N >= W else N * (N + 1) // 2
+        self.flops = 4 * d * pairs * Hq * B
+        self.tail = min(N, W)
+
+    def step(self, ev=None):
+        hs = self.hs
+        if ev is not None:
+            ev[0].record()
+        hs.swa_prefill_fwd(self.pool, 0, self.q, self.k, self.v, o=self.o)
+        if ev is not None:
+            ev[1].record()
+        # commit the chunk into the rolling buffer (only its last W tokens land)
+        hs.kv_pool_append(self.pool, 0, self.k, self.v, self.start, seq_ids=self.seq_ids)
+
+    launches_per_step = 2
+
+    def e2e_setup(self):
+        self.hq = self.q.cpu().pin_memory()
+        self.hk = self.k.cpu().pin_memory()
+        self.hv = self.v.cpu().pin_memory()
+        self.ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = (self.hq.numel() + self.hk.numel() + self.hv.numel()) * 2
+        self.d2h = self.ho.numel() * 2
+
+    def e2e_step(self):
+        self.q.copy_(self.hq, non_blocking=True)
+        self.k.copy_(self.hk, non_blocking=True)
+        self.v.copy_(self.hv, non_blocking=True)
+        self.step()
+        self.ho.copy_(self.o, non_blocking=True)
+
+    def check_sample(self, oracle, rows=(0, 1, 127, 128, 4095, 4096, 9999, 16383)):
+        """Sampled rows (all heads, both sequences) against the oracle; returns (max, mean) abs error."""
+        errs = []
+        for b in range(self.B):
+            lo = max(0, min(rows) - self.W + 1)
+            hi = max(rows) + 1
+            k = gen(synth.TAG_K, 0, self.seq_offset + b, lo, hi - lo, self.Hkv, self.d, self.sigma, "cpu")
+            v = gen(synth.TAG_V, 0, self.seq_offset + b, lo, hi - lo, self.Hkv, self.d, self.sigma, "cpu")
+            qr = torch.stack([gen(synth.TAG_Q, 0, self.seq_offset + b, r, 1, self.Hq, self.d, self.sigma, "cpu")[0]
+                              for r in rows])
+            ref = oracle.attention(qr, np.array(rows), k, v, self.W, key_base=lo)
+            got = self.o[b, list(rows)].float().cpu().double().numpy()
+            errs.append(np.abs(got - ref))
+        e = np.concatenate([x.ravel() for x in errs])
+        return float(e.max()), float(e.mean())
+
+    def oracle_sample(self, oracle, budget_s=10.0, block=32, threads=None):
+        """Time the oracle on blocks of query rows (all heads, full W-key windows) taken from the end of
+        sequence 0 until about budget_s seconds have passed; returns (seconds, flops, rows)."""
+        max_rows = 2048
+        rows_all = np.arange(self.N - max_rows, self.N)
+        lo = rows_all[0] - self.W + 1
+        k = gen(synth.TAG_K, 0, self.seq_offset, lo, self.N - lo, self.Hkv, self.d, self.sigma, "cpu")
+        v = gen(synth.TAG_V, 0, self.seq_offset, lo, self.N - lo, self.Hkv, self.d, self.sigma, "cpu")
+        q = gen(synth.TAG_Q, 0, self.seq_offset, rows_all[0], max_rows, self.Hq, self.d, self.sigma, "cpu")
+        done, dt = 0, 0.0
+        while dt < budget_s and done < max_rows:
+            r = rows_all[done:done + block]
+            t0 = time.perf_counter()
+            oracle.attention(q[done:done + block], r, k, v, self.W, key_base=lo, n_threads=threads)
+            dt += time.perf_counter() - t0
+            done += len(r)
+        flops = 4 * self.d * done * self.W * self.Hq
+        return dt, flops, done
+
+
+def time_region(fn, steps, stream, ev_pairs=None):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(ev_pairs[i] if ev_pairs else None)
+    e1.record(stream)
+    return e0, e1
+
+
+def secondary_results(hs, oracle_mod, hbm, bf16):
+    out = []
+    dev = "cuda"
+
+    def t(fn, reps, warm=3):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    # config 1: B=1, N=512, Hq=4, Hkv=1, d=64, W in {128, 512, 1}
+    for W in (128, 512, 1):
+        pool = hs.kv_pool_create(hs.PoolDesc(1, 0, W, 1, 64, 1, 0))
+        q = gen(synth.TAG_Q, 10, 0, 0, 512, 4, 64, 1.0, dev)[None]
+        k = gen(synth.TAG_K, 10, 0, 0, 512, 1, 64, 1.0, dev)[None]
+        v = gen(synth.TAG_V, 10, 0, 0, 512, 1, 64, 1.0, dev)[None]
+        o = torch.empty_like(q)
+        ms = t(lambda: hs.swa_prefill_fwd(pool, 0, q, k, v, o=o), 50)
+        kk = gen(synth.TAG_K, 10, 0, 0, 512, 1, 64, 1.0, "cpu")
+        vv = gen(synth.TAG_V, 10, 0, 0, 512, 1, 64, 1.0, "cpu")
+        qq = gen(synth.TAG_Q, 10, 0, 0, 512, 4, 64, 1.0, "cpu")
+        ref = oracle_mod.attention(qq, np.arange(512), kk, vv, W)
+        err = np.abs(o[0].float().cpu().double().numpy() - ref)
+        out.append({"workload": f"swa_layer_512_W{W}_Hq4_Hkv1_d64", "metric": "latency", "unit": "us",
+                    "value": round(ms * 1000, 2), "max_abs_err": float(err.max()), "mean_abs_err": float(err.mean())})
+
+    # config 3: 16K chunk after a 131072-token prefix; SWA layer W=128 (ring) + full layer (pages)
+    P, Nc, Hq, Hkv, d, W = 131072, 16384, 64, 8, 128, 128
+    total = P + Nc
+    pages = total // 64
+    pool = hs.kv_pool_create(hs.PoolDesc(1, 1, W, Hkv, d, 1, pages))
+    perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 3), pages).to(torch.int32)
+    pt = perm.view(1, pages).to(dev)
+    sid = torch.zeros(1, dtype=torch.int32, device=dev)
+    sp = torch.tensor([P], dtype=torch.int64, device=dev)
+    kp = gen(synth.TAG_K, 0, 100, P - W, W, Hkv, d, 1.0, dev)[None]
+    vp = gen(synth.TAG_V, 0, 100, P - W, W, Hkv, d, 1.0, dev)[None]
+    hs.kv_pool_append(pool, 0, kp, vp, torch.tensor([P - W], device=dev), seq_ids=sid)
+    for c0 in range(0, total, 16384):
+        n = min(16384, total - c0)
+        kf = gen(synth.TAG_K, 1, 100, c0, n, Hkv, d, 1.0, dev)[None]
+        vf = gen(synth.TAG_V, 1, 100, c0, n, Hkv, d, 1.0, dev)[None]
+        hs.kv_pool_append(pool, 1, kf, vf, torch.tensor([c0], device=dev), page_table=pt)
+    q0 = gen(synth.TAG_Q, 0, 100, P, Nc, Hq, d, 1.0, dev)[None]
+    k0 = gen(synth.TAG_K, 0, 100, P, Nc, Hkv, d, 1.0, dev)[None]
+    v0 = gen(synth.TAG_V, 0, 100, P, Nc, Hkv, d, 1.0, dev)[None]
+    q1 = gen(synth.TAG_Q, 1, 100, P, Nc, Hq, d, 1.0, dev)[None]
+    o0 = torch.empty_like(q0)
+    o1 = torch.empty_like(q1)
+    ms_swa = t(lambda: hs.swa_prefill_fwd(pool, 0, q0, k0, v0, o=o0, start_pos=sp, seq_ids=sid), 20)
+    ms_full = t(lambda: hs.full_prefill_fwd(pool, 1, q1, pt, o=o1, start_pos=sp), 3, warm=1)
+    swa_flops = 4 * d * Nc * W * Hq
+    swa_bytes = (2 * Nc * Hq * d + 2 * Nc * Hkv * d + 2 * W * Hkv * d) * 2
+    full_flops = 4 * d * (Nc * P + Nc * (Nc + 1) // 2) * Hq
+    rows = [0, 1, 127, 128, 8191, 16383]
+    qq = gen(synth.TAG_Q, 0, 100, P, Nc, Hq, d, 1.0, "cpu")[rows]
+    kk = gen(synth.TAG_K, 0, 100, P - W + 1, Nc + W - 1, Hkv, d, 1.0, "cpu")
+    vv = gen(synth.TAG_V, 0, 100, P - W + 1, Nc + W - 1, Hkv, d, 1.0, "cpu")
+    e_swa = np.abs(o0[0, rows].float().cpu().double().numpy() -
+                   oracle_mod.attention(qq, P + np.array(rows), kk, vv, W, key_base=P - W + 1))
+    rows_f = [0, 16383]
+    qf = gen(synth.TAG_Q, 1, 100, P, Nc, Hq, d, 1.0, "cpu")[rows_f]
+    kf = gen(synth.TAG_K, 1, 100, 0, total, Hkv, d, 1.0, "cpu")
+    vf = gen(synth.TAG_V, 1, 100, 0, total, Hkv, d, 1.0, "cpu")
+    e_full = np.abs(o1[0, rows_f].float().cpu().double().numpy() -
+                    oracle_mod.attention(qf, P + np.array(rows_f), kf, vf, 0))
+    out.append({"workload": "hybrid_chunk16k_after_131072_swa_W128_Hq64_Hkv8_d128", "metric": "KV+Q+O GB/s",
+                "unit": "GB/s", "value": round(swa_bytes / ms_swa / 1e6, 1), "ms": round(ms_swa, 4),
+                "tflops": round(swa_flops / ms_swa / 1e9, 1), "pct_hbm_peak": round(100 * swa_bytes / ms_swa / 1e6 / hbm, 1),
+                "max_abs_err": float(e_swa.max()), "mean_abs_err": float(e_swa.mean())})
+    out.append({"workload": "hybrid_chunk16k_after_131072_full_paged_Hq64_Hkv8_d128", "metric": "prefill TFLOP/s",
+                "unit": "TFLOP/s", "value": round(full_flops / ms_full / 1e9, 1), "ms": round(ms_full, 3),
+                "pct_bf16_peak": round(100 * full_flops / ms_full / 1e9 / bf16, 1),
+                "max_abs_err": float(e_full.max()), "mean_abs_err": float(e_full.mean())})
+    del pool, q0, k0, v0, q1, o0, o1
+    torch.cuda.empty_cache()
+
+    # config 4: decode batch
+    out.extend(decode_results(hs, oracle_mod, hbm))
+    return out
+
+
+def decode_results(hs, oracle_mod, hbm):
+    dev = "cuda"
+    n, Hq, Hkv, d, W, nq = 256, 64, 8, 128, 128, 4
+    u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 4), n)
+    lens = torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
+    S = int(lens.sum())
+    pps = (lens + nq + 63) // 64
+    total_pages = int(pps.sum())
+    maxp = int(pps.max())
+    n_swa = 6
+    pool = hs.kv_pool_create(hs.PoolDesc(n_swa, 1, W, Hkv, d, n, total_pages))
+    perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 5), total_pages).to(torch.int32)
+    pt = torch.zeros(n, maxp, dtype=torch.int32)
+    off = 0
+    for i in range(n):
+        pt[i, :pps[i]] = perm[off:off + int(pps[i])]
+        off += int(pps[i])
+    pt = pt.to(dev)
+    sid = torch.arange(n, dtype=torch.int32, device=dev)
+    full_layer = n_swa
+    for b in range(n):
+        L = int(lens[b])
+        for c0 in range(0, L, 65536):
+            m = min(65536, L - c0)
+            k = gen(synth.TAG_K, full_layer, 200 + b, c0, m, Hkv, d, 1.0, dev)[None]
+            v = gen(synth.TAG_V, full_layer, 200 + b, c0, m, Hkv, d, 1.0, dev)[None]
+            hs.kv_pool_append(pool, full_layer, k, v, torch.tensor([c0], device=dev), page_table=pt[b:b + 1])
+        for layer in range(n_swa):
+            k = gen(synth.TAG_K, layer, 200 + b, L - W, W, Hkv, d, 1.0, dev)[None]
+            v = gen(synth.TAG_V, layer, 200 + b, L - W, W, Hkv, d, 1.0, dev)[None]
+            hs.kv_pool_append(pool, layer, k, v, torch.tensor([L - W], device=dev), seq_ids=sid[b:b + 1])
+    ctx = lens.to(dev)
+    maxL = int(lens.max())
+    qs, kn, vn = [], [], []
+    for layer in range(n_swa + 1):
+        qs.append(torch.stack([gen(synth.TAG_Q, layer, 200 + b, int(lens[b]), nq, Hq, d, 1.0, dev) for b in range(n)]))
+        kn.append(torch.stack([gen(synth.TAG_K, layer, 200 + b, int(lens[b]), nq, Hkv, d, 1.0, dev) for b in range(n)]))
+        vn.append(torch.stack([gen(synth.TAG_V, layer, 200 + b, int(lens[b]), nq, Hkv, d, 1.0, dev) for b in range(n)]))
+    ws = torch.empty(hs.hybrid_decode_workspace_size(pool, n, nq, Hq, maxL), dtype=torch.uint8, device=dev)
+    outs = [torch.empty_like(qs[0]) for _ in range(n_swa + 1)]
+
+    def step():
+        for layer in range(n_swa):
+            hs.hybrid_decode_fwd(pool, layer, qs[layer], kn[layer], vn[layer], ctx, maxL, ws, seq_ids=sid,
+                                 o=outs[layer])
+        hs.hybrid_decode_fwd(pool, full_layer, qs[n_swa], kn[n_swa], vn[n_swa], ctx, maxL, ws, page_table=pt,
+                             o=outs[n_swa])
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    times, times_full = [], []
+    for _ in range(5):
+        flush.zero_()
+        a, b_, c = (torch.cuda.Event(True) for _ in range(3))
+        a.record()
+        for layer in range(n_swa):
+            hs.hybrid_decode_fwd(pool, layer, qs[layer], kn[layer], vn[layer], ctx, maxL, ws, seq_ids=sid,
+                                 o=outs[layer])
+        b_.record()
+        hs.hybrid_decode_fwd(pool, full_layer, qs[n_swa], kn[n_swa], vn[n_swa], ctx, maxL, ws, page_table=pt,
+                             o=outs[n_swa])
+        c.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(c))
+        times_full.append(b_.elapsed_time(c))
+    ms = statistics.median(times)
+    ms_full = statistics.median(times_full)
+    kv_full = S * Hkv * d * 2 * 2
+    kv_swa = n_swa * n * (W - 1) * Hkv * d * 2 * 2
+    qo = (n_swa + 1) * n * nq * (Hq * 2 + Hkv * 2) * d * 2
+    total_bytes = kv_full + kv_swa + qo
+    assert hs.hswa_pool_check_error(pool) == 0
+    # sampled parity: the two shortest sequences (full layer) and two sequences of one SWA layer
+    order = torch.argsort(lens)
+    errs = []
+    for b in [int(order[0]), int(order[1])]:
+        L = int(lens[b])
+        k = gen(synth.TAG_K, full_layer, 200 + b, 0, L + nq, Hkv, d, 1.0, "cpu")
+        v = gen(synth.TAG_V, full_layer, 200 + b, 0, L + nq, Hkv, d, 1.0, "cpu")
+        q = gen(synth.TAG_Q, full_layer, 200 + b, L, nq, Hq, d, 1.0, "cpu")
+        ref = oracle_mod.attention(q, L + np.arange(nq), k, v, 0)
+        errs.append(np.abs(outs[n_swa][b].float().cpu().double().numpy() - ref).ravel())
+    for b in [int(order[-1]), 7]:
+        L = int(lens[b])
+        k = gen(synth.TAG_K, 2, 200 + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
+        v = gen(synth.TAG_V, 2, 200 + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
+        q = gen(synth.TAG_Q, 2, 200 + b, L, nq, Hq, d, 1.0, "cpu")
+        ref = oracle_mod.attention(q, L + np.arange(nq), k, v, W, key_base=L - W + 1)
+        errs.append(np.abs(outs[2][b].float().cpu().double().numpy() - ref).ravel())
+    e = np.concatenate(errs)
+    res = [{"workload": "hybrid_decode_256seq_L1K-256K_6swa_1full_Hq64_Hkv8_d128_4tok", "metric": "hybrid decode KV GB/s",
+            "unit": "GB/s", "value": round(total_bytes / ms / 1e6, 1), "ms": round(ms, 3),
+            "pct_hbm_peak": round(100 * total_bytes / ms / 1e6 / hbm, 1), "bytes": total_bytes, "sum_ctx": S,
+            "full_layer_ms": round(ms_full, 3), "full_layer_gbs": round((kv_full + qo / 7) / ms_full / 1e6, 1),
+            "l2": "flushed (256 MiB write) before each step", "max_abs_err": float(e.max()),
+            "mean_abs_err": float(e.mean())}]
+    # window_safe_len over 4096 requests (bit-exact vs oracle)
+    nr = 4096
+    C = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 11), nr, 0, 262144)
+    M = torch.where(synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 12), nr, 0, 1) == 0, C,
+                    synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 13), nr, 0, 262144))
+    # masks: half all-valid, a quarter with one random evicted slot, a quarter with slot C mod W evicted
+    bits = np.full((nr, W // 32), 0xFFFFFFFF, dtype=np.uint32)
+    ev = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 14), nr, 0, W - 1).numpy()
+    kind = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 15), nr, 0, 3).numpy()
+    for r in range(nr):
+        s = int(C[r]) % W if kind[r] == 3 else (int(ev[r]) if kind[r] == 2 else -1)
+        if s >= 0:
+            bits[r, s // 32] &= np.uint32(~(1 << (s % 32)) & 0xFFFFFFFF)
+    Md, Cd, Bd = M.to(dev), C.to(dev), torch.from_numpy(bits.view(np.int32)).to(dev)
+    outw = torch.empty(nr, dtype=torch.int64, device=dev)
+    for _ in range(5):
+        hs.window_safe_len(Md, Cd, Bd, W, out=outw)
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(True), torch.cuda.Event(True)
+    a.record()
+    for _ in range(100):
+        hs.window_safe_len(Md, Cd, Bd, W, out=outw)
+    b_.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b_) / 100 * 1000
+    ref = oracle_mod.window_safe_len(M.numpy(), C.numpy(), bits, W)
+    res.append({"workload": "window_safe_len_4096req_W128", "metric": "latency", "unit": "us", "value": round(us, 2),
+                "requests_per_s": round(nr / (us * 1e-6)), "bit_exact": bool(np.array_equal(outw.cpu().numpy(), ref))})
+    del pool
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    B, N, W, Hq, Hkv, d = 2, 16384, 4096, 32, 8, 128
+    sigma = 2 ** -0.5
+    n_rows = 32
+    rows = np.arange(N - n_rows, N)
+    lo = rows[0] - W + 1
+    k = gen(synth.TAG_K, 0, 0, lo, N - lo, Hkv, d, sigma, "cpu")
+    v = gen(synth.TAG_V, 0, 0, lo, N - lo, Hkv, d, sigma, "cpu")
+    q = gen(synth.TAG_Q, 0, 0, rows[0], n_rows, Hq, d, sigma, "cpu")
+    for _ in range(args.warmup):
+        oracle.attention(q, rows, k, v, W, key_base=lo, n_threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention(q, rows, k, v, W, key_base=lo, n_threads=threads)
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 4 * d * n_rows * W * Hq
+    val = flops / dt / 1e12
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1000, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": SwaPrefill16k.name, "B": B, "N": N, "W": W, "Hq": Hq, "Hkv": Hkv, "head_dim": d},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n_rows} query rows x {Hq} heads at the end of sequence 0 (full W-key windows) per step"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hswa", choices=["hswa", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    ws, rank, local = dist_setup() if args.impl == "hswa" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        return
+
+    torch.cuda.set_device(local)
+    import hybrid_sliding_window_swa_b200 as hs
+    hs.load_library()
+    hbm, bf16, bf16_sus, peak_src = peaks()
+    wl = SwaPrefill16k(hs, seq_offset=rank * 2)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    assert hs.hswa_pool_check_error(wl.pool) == 0
+
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    e0, e1 = time_region(wl.step, args.steps, stream, ev_pairs)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in ev_pairs) / args.steps
+    ms_max = max_over_ranks(ms_step, ws)
+    value = wl.flops * ws / ms_max / 1e9  # TFLOP/s over all ranks
+    achieved = wl.flops / kern_ms / 1e9
+
+    max_err, mean_err = (None, None)
+    e2e = None
+    cpu = None
+    sec = None
+    if not args.no_e2e:
+        wl.e2e_setup()
+        for _ in range(2):
+            wl.e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+        a.record()
+        for _ in range(max(3, args.steps // 4)):
+            wl.e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / max(3, args.steps // 4), ws)
+        e2e = {"value": round(wl.flops * ws / e2e_ms / 1e9, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+               "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
+               "path": "pinned host Q/K/V -> device, swa_prefill_fwd + kv_pool_append via the Python binding "
+                       "(C ABI), O -> pinned host"}
+    if rank == 0:
+        import oracle
+        oracle.build()
+        max_err, mean_err = wl.check_sample(oracle)
+        if not args.no_cpu:
+            threads = os.cpu_count() or 1
+            dt, fl, nrows = wl.oracle_sample(oracle, threads=threads)
+            cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                   "sample": f"{nrows} query rows x 32 heads at the end of sequence 0 (full 4096-key windows), "
+                             f"fp64, {dt:.1f} s"}
+        if not args.no_secondary and ws == 1:
+            sec = secondary_results(hs, oracle, hbm, bf16)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based N(0,1/2) bf16)",
+            "config": {"workload": wl.name, "B_per_gpu": wl.B, "seq_len": wl.N, "window": wl.W, "Hq": wl.Hq,
+                       "Hkv": wl.Hkv, "head_dim": wl.d, "parallelism": f"independent batches x{ws}",
+                       "step": "swa_prefill_fwd + kv_pool_append(ring commit)",
+                       "l2": "inputs larger than L2 (Q 268 MB + K/V 134 MB + O 268 MB per step)"},
+            "pct_bf16_peak": round(100 * value / ws / bf16, 1),
+            "roofline": {"bound": "tensor", "kernel": "prefill_kernel<128> (swa_prefill_fwd)",
+                         "achieved": round(achieved, 1), "peak": bf16, "unit": "TFLOP/s",
+                         "frac": round(achieved / bf16, 3), "peak_source": f"{peak_src} bf16 burst",
+                         "algorithmic_flops_per_launch": wl.flops, "kernel_ms": round(kern_ms, 4),
+                         "traffic": None},
+            "parity": {"max_abs_err": max_err, "mean_abs_err": mean_err, "rows": "8 rows x 32 heads x 2 seqs"},
+            "gpu_launches": wl.launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        if e2e:
+            line["e2e"] = e2e
+        if sec:
+            line["secondary"] = sec
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

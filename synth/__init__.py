@@ -140,11 +140,45 @@ def _table_on(sigma: float, device: torch.device):
     return _DEV_TABLES[key]
 
 
+_FAST = None
+
+
+def _fast_lib():
+    """The C build of the same generator (CPU only); None if gcc is unavailable."""
+    global _FAST
+    if _FAST is None:
+        import ctypes
+        import os
+        import subprocess
+        here = os.path.dirname(os.path.abspath(__file__))
+        src, lib = os.path.join(here, "fastgen.c"), os.path.join(here, "libfastgen.so")
+        try:
+            if not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+                tmp = lib + f".tmp{os.getpid()}"
+                subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-pthread", "-o", tmp, src])
+                os.replace(tmp, lib)
+            L = ctypes.CDLL(lib)
+            L.fastgen_normal_bf16.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                              ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+            L.fastgen_normal_bf16.restype = ctypes.c_int
+            _FAST = L
+        except Exception:  # pragma: no cover - torch path below still works
+            _FAST = False
+    return _FAST or None
+
+
 def normal_bf16(seed: int, stream: int, start: int, count: int, sigma: float = 1.0,
-                device="cpu", chunk: int = 1 << 26) -> torch.Tensor:
+                device="cpu", chunk: int = 1 << 26, use_c: bool = True) -> torch.Tensor:
     """``count`` bf16 values: draws ``start .. start+count-1`` of (seed, stream), N(0, sigma^2)."""
     device = torch.device(device)
     key = stream_key(seed, stream)
+    if device.type == "cpu" and use_c and count >= 4096 and _fast_lib() is not None:
+        import os
+        thr, val = normal_table(float(sigma))
+        out = torch.empty(count, dtype=torch.int16)
+        _fast_lib().fastgen_normal_bf16(key, start, count, thr.data_ptr(), thr.numel(), val.data_ptr(),
+                                        out.data_ptr(), os.cpu_count() or 1)
+        return out.view(torch.bfloat16)
     thr, val = _table_on(float(sigma), device)
     out = torch.empty(count, dtype=torch.int16, device=device)
     for c0 in range(0, count, chunk):

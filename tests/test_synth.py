@@ -44,3 +44,11 @@ def test_uniform_int_range_and_permutation():
     assert int(u.min()) == 5 and int(u.max()) == 17
     p = synth.permutation(3, synth.stream_id(synth.TAG_MISC, 1), 1000)
     assert sorted(p.tolist()) == list(range(1000))
+
+
+def test_c_and_torch_generators_agree_bitwise():
+    s = synth.stream_id(synth.TAG_K, 1, 2)
+    for sigma in (1.0, 2 ** -0.5):
+        a = synth.normal_bf16(5, s, 1000, 300_000, sigma, use_c=False)
+        b = synth.normal_bf16(5, s, 1000, 300_000, sigma, use_c=True)
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
