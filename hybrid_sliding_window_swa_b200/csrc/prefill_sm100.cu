@@ -10,15 +10,20 @@
 // Attention and BlockSparse": blocks outside the window are skipped); only tiles
 // that the band edge crosses are masked.
 //
-// CTA = 2 query tiles of 128 rows (one batch row b, one query head h).
-//   warp 0      producer: Q once, then K/V tiles into a 2-stage ring of shared-memory
-//               buffers (TMA for chunk rows and pages; cp.async for rolling-buffer
-//               rows that are not 128-aligned).
-//   warp 1      MMA issuer (one thread): S_q = Q_q K_j^T into TMEM, O_q += P_q V_j
+// Work unit = 2 query tiles of 128 rows (one batch row b, one query head h). The grid
+// is persistent (one CTA per SM) and walks the units in a static round-robin, heaviest
+// (latest query tiles) first; consecutive CTAs take the query heads of one KV group
+// so their K/V tiles are shared through L2.
+//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one thread per
+//               row (TMEM lane); all 128 scores of a row in registers, online max/sum
+//               in the exp2 domain with lazy O rescaling, exponentials split between
+//               the MUFU unit and an FMA-pipe polynomial, P written back over S as
+//               packed bf16, and the epilogue (O / l -> bf16 -> global).
+//   warp 8      producer: Q of each unit, then K/V tiles into a 2-stage ring of
+//               shared-memory buffers (TMA for chunk rows, aligned ring tiles and
+//               pages; cp.async for rolling-buffer rows that are not 128-aligned).
+//   warp 9      MMA issuer (one thread): S_q = Q_q K_j^T into TMEM, O_q += P_q V_j
 //               with P_q read from TMEM; also allocates/frees TMEM.
-//   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1: one thread per
-//               row (TMEM lane), online max/sum in the exp2 domain with lazy O
-//               rescaling, P written back over S as packed bf16, and the epilogue.
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
 //
 // Key tiles. Sliding-window layers: tile j covers positions [P + 128 j, P + 128 j + 128)
@@ -34,10 +39,14 @@ namespace {
 
 constexpr int BM = 128;     // query rows per tile
 constexpr int BN = 128;     // keys per tile
-constexpr int NQT = 2;      // query tiles per CTA
+constexpr int NQT = 2;      // query tiles per unit
 constexpr int NSTAGE = 2;   // K/V pipeline depth
-constexpr int NTHREADS = 384;
+constexpr int NWARPS = 10;
+constexpr int NTHREADS = NWARPS * 32;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
 constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <= 2^8
+constexpr int kPolyEvery = 4; // one pair in kPolyEvery takes the FMA-pipe exponential
 
 struct Params {
   int B, n_q, Hq, Hkv, G;
@@ -55,6 +64,8 @@ struct Params {
   int64_t pages;
   float scale_log2;
   int n_pairs;
+  int n_units;
+  int64_t max_start;  // largest start position that keeps every position below 2^31
   int* err;
 };
 
@@ -72,48 +83,59 @@ struct Layout {
 };
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE];
   uint64_t s_full[NQT], p_full[NQT], o_full[NQT];
   uint64_t v_fix;  // TMA completion of the page tile that holds the last key (before its tail is zeroed)
   uint32_t tmem_base;
 };
 
-// Geometry of one CTA's work, computed identically by every role.
+// Geometry of one work unit, computed identically by every role.
+// Positions are below 2^31 (checked on the host against start_pos bounds on the device).
 struct Geo {
   int b, h, g;
-  int64_t P;             // absolute position of the chunk's first row
+  int P;                 // absolute position of the chunk's first row
   int t[NQT];            // query tile index within the chunk
   bool act[NQT];
-  int64_t i0[NQT], i1[NQT];  // first / last valid absolute query position of each tile
-  int64_t jlo[NQT], jhi[NQT];
-  int64_t jb, je;        // union of needed key tiles, inclusive
+  int i0[NQT], i1[NQT];  // first / last valid absolute query position of each tile
+  int jlo[NQT], jhi[NQT];
+  int jb, je;            // union of needed key tiles, inclusive
 };
 
-__device__ __forceinline__ int64_t window_lo(const Params& p, int64_t i) {
+__device__ __forceinline__ int window_lo(const Params& p, int i) {
   if (p.window <= 0) return 0;
-  const int64_t lo = i - p.window + 1;
+  const int lo = i - p.window + 1;
   return lo > 0 ? lo : 0;
 }
 
-__device__ __forceinline__ int64_t key_base(const Params& p, const Geo& G, int64_t j) {
-  return p.is_full ? (int64_t)BN * j : G.P + (int64_t)BN * j;
+__device__ __forceinline__ int key_base(const Params& p, const Geo& G, int j) {
+  return p.is_full ? BN * j : G.P + BN * j;
 }
 
-__device__ __forceinline__ void make_geo(const Params& p, Geo& G) {
-  G.h = blockIdx.x;
-  const int pair = p.n_pairs - 1 - (int)blockIdx.y;  // longest causal work first
-  G.b = blockIdx.z;
+__device__ __forceinline__ void make_geo(const Params& p, int unit, Geo& G) {
+  const int per_pair = p.B * p.Hq;
+  const int pair = p.n_pairs - 1 - unit / per_pair;  // latest (longest causal) tiles first
+  const int rem = unit % per_pair;
+  G.b = rem / p.Hq;
+  G.h = rem % p.Hq;
   G.g = G.h / p.G;
-  G.P = p.start_pos ? p.start_pos[G.b] : 0;
-  G.jb = INT64_MAX;
-  G.je = INT64_MIN;
+  int64_t P = p.start_pos ? p.start_pos[G.b] : 0;
+  if (P < 0 || P > p.max_start) {  // positions must stay below 2^31
+    record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+    P = 0;
+  }
+  G.P = (int)P;
+  G.jb = INT32_MAX;
+  G.je = INT32_MIN;
+#pragma unroll
   for (int q = 0; q < NQT; ++q) {
     G.t[q] = pair * NQT + q;
-    const int64_t r0 = (int64_t)G.t[q] * BM;
+    const int r0 = G.t[q] * BM;
     G.act[q] = r0 < p.n_q;
+    G.i0[q] = G.i1[q] = G.jlo[q] = 0;
+    G.jhi[q] = -1;
     if (!G.act[q]) continue;
-    const int64_t r1 = (r0 + BM - 1 < p.n_q - 1) ? r0 + BM - 1 : p.n_q - 1;
+    const int r1 = (r0 + BM - 1 < p.n_q - 1) ? r0 + BM - 1 : p.n_q - 1;
     G.i0[q] = G.P + r0;
     G.i1[q] = G.P + r1;
     if (p.is_full) {
@@ -128,13 +150,13 @@ __device__ __forceinline__ void make_geo(const Params& p, Geo& G) {
   }
 }
 
-__device__ __forceinline__ bool needs(const Geo& G, int q, int64_t j) {
+__device__ __forceinline__ bool needs(const Geo& G, int q, int j) {
   return G.act[q] && j >= G.jlo[q] && j <= G.jhi[q];
 }
 
 // All (row, key) pairs of the tile are inside the band.
-__device__ __forceinline__ bool mask_free(const Params& p, const Geo& G, int q, int64_t j) {
-  const int64_t kb = key_base(p, G, j);
+__device__ __forceinline__ bool mask_free(const Params& p, const Geo& G, int q, int j) {
+  const int kb = key_base(p, G, j);
   return kb + BN - 1 <= G.i0[q] && kb >= window_lo(p, G.i1[q]);
 }
 
@@ -144,18 +166,18 @@ __device__ __forceinline__ bool mask_free(const Params& p, const Geo& G, int q, 
 // rows whose position is not held by the ring (or is negative) are zero-filled.
 template <int D>
 __device__ __forceinline__ void ring_tile_cpasync(const Params& p, const Geo& G, const uint16_t* ring,
-                                                  uint8_t* dst, int64_t kb, int lane) {
+                                                  uint8_t* dst, int kb, int lane) {
   const int seq = p.seq_ids ? p.seq_ids[G.b] : 0;
   const bool seq_ok = seq >= 0 && seq < p.max_seqs;
   if (!seq_ok && lane == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
   const int64_t row_base = seq_ok ? (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + G.g) * p.window : 0;
-  const int64_t held_lo = (G.P - p.window > 0) ? G.P - p.window : 0;
+  const int held_lo = (G.P - p.window > 0) ? G.P - p.window : 0;
   const uint32_t sdst = smem_u32(dst);
   constexpr int CH = D / 8;  // 16-byte chunks per row
   for (int idx = lane; idx < BN * CH; idx += 32) {
     const int r = idx / CH;
     const int c = idx % CH;
-    const int64_t pos = kb + r;
+    const int pos = kb + r;
     const bool held = seq_ok && pos >= held_lo && pos < G.P;
     const uint16_t* src = ring + (held ? (row_base + (pos % p.window)) * D + c * 8 : 0);
     const int blk = c >> 3, cc = c & 7;
@@ -168,101 +190,112 @@ __device__ __forceinline__ void ring_tile_cpasync(const Params& p, const Geo& G,
 }
 
 template <int D>
-__device__ void producer(const Params& p, const Geo& G, uint8_t* smem, Bars* bars, const CUtensorMap* tm_q,
+__device__ void producer(const Params& p, uint8_t* smem, Bars* bars, const CUtensorMap* tm_q,
                          const CUtensorMap* tm_k, const CUtensorMap* tm_v, const CUtensorMap* tm_rk,
                          const CUtensorMap* tm_rv) {
   using L = Layout<D>;
   const int lane = threadIdx.x & 31;
-  if (lane == 0) {
-    int nact = 0;
-    for (int q = 0; q < NQT; ++q) nact += G.act[q];
-    mbar_arrive_expect_tx(&bars->q_full, nact * L::TILE);
-    for (int q = 0; q < NQT; ++q) {
-      if (!G.act[q]) continue;
-      for (int dh = 0; dh < D / 64; ++dh)
-        tma_load_4d(smem + L::Q_OFF + q * L::TILE + dh * L::BLOCK, tm_q, &bars->q_full, dh * 64, G.h,
-                    G.t[q] * BM, G.b);
+  int it = 0;        // K/V tiles loaded so far (stage ring position)
+  uint32_t uq = 0;   // units started (Q buffer phase)
+  uint32_t nfix = 0; // page tiles zero-filled past the last key (v_fix phase)
+  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++uq) {
+    Geo G;
+    make_geo(p, unit, G);
+    // the Q buffers are free once every S MMA of the previous unit has completed
+    if (!mbar_wait(&bars->q_empty, (uq & 1) ^ 1, p.err)) return;
+    if (lane == 0) {
+      int nact = 0;
+      for (int q = 0; q < NQT; ++q) nact += G.act[q];
+      mbar_arrive_expect_tx(&bars->q_full, nact * L::TILE);
+      for (int q = 0; q < NQT; ++q) {
+        if (!G.act[q]) continue;
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_4d(smem + L::Q_OFF + q * L::TILE + dh * L::BLOCK, tm_q, &bars->q_full, dh * 64, G.h,
+                      G.t[q] * BM, G.b);
+      }
     }
-  }
-  // highest key position any query of this CTA may need
-  int64_t kmax = 0;
-  for (int q = 0; q < NQT; ++q)
-    if (G.act[q] && G.i1[q] > kmax) kmax = G.i1[q];
-  const int seq = (!p.is_full && p.seq_ids) ? p.seq_ids[G.b] : 0;
-  const bool ring_fast = p.ring_tma && (G.P % BN) == 0;
+    __syncwarp();
+    // highest key position any query of this unit may need
+    int kmax = 0;
+    for (int q = 0; q < NQT; ++q)
+      if (G.act[q] && G.i1[q] > kmax) kmax = G.i1[q];
+    const int seq = (!p.is_full && p.seq_ids) ? p.seq_ids[G.b] : 0;
+    const bool ring_fast = p.ring_tma && (G.P % BN) == 0;
 
-  int it = 0;
-  for (int64_t j = G.jb; j <= G.je; ++j, ++it) {
-    const int s = it % NSTAGE;
-    const uint32_t ph = (it / NSTAGE) & 1;
-    const int64_t kb = key_base(p, G, j);
-    for (int kv = 0; kv < 2; ++kv) {
-      uint64_t* full = kv ? &bars->v_full[s] : &bars->k_full[s];
-      uint64_t* empty = kv ? &bars->v_empty[s] : &bars->k_empty[s];
-      uint8_t* dst = smem + (kv ? L::V_OFF : L::K_OFF) + s * L::TILE;
-      if (!mbar_wait(empty, ph ^ 1, p.err)) return;
-      if (p.is_full) {
-        // Rows of the last page past the last key hold stale memory; P is 0 there, but
-        // 0 * NaN would still poison P V, so that V tile is zeroed past kmax before use.
-        const bool fix = kv == 1 && kb <= kmax && kmax < kb + BN - 1 && ((kmax + 1) % 64) != 0;
-        uint64_t* land = fix ? &bars->v_fix : full;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(land, L::TILE);
-          const CUtensorMap* tm = kv ? tm_v : tm_k;
-          for (int half = 0; half < 2; ++half) {
-            const int64_t pos0 = kb + 64 * half;
-            const int64_t lp = pos0 / 64;
-            int64_t row = -1;  // outside the map: zero fill
-            if (pos0 <= kmax) {
-              int32_t page = -1;
-              if (lp < p.pt_stride) page = p.page_table[(int64_t)G.b * p.pt_stride + lp];
-              if (page < 0 || page >= p.pages) {
-                record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
-              } else {
-                row = ((int64_t)p.full_layer * p.pages + page) * p.Hkv + G.g;
+    for (int j = G.jb; j <= G.je; ++j, ++it) {
+      const int s = it % NSTAGE;
+      const uint32_t ph = (it / NSTAGE) & 1;
+      const int kb = key_base(p, G, j);
+      for (int kv = 0; kv < 2; ++kv) {
+        uint64_t* full = kv ? &bars->v_full[s] : &bars->k_full[s];
+        uint64_t* empty = kv ? &bars->v_empty[s] : &bars->k_empty[s];
+        uint8_t* dst = smem + (kv ? L::V_OFF : L::K_OFF) + s * L::TILE;
+        if (!mbar_wait(empty, ph ^ 1, p.err)) return;
+        if (p.is_full) {
+          // Rows of the last page past the last key hold stale memory; P is 0 there, but
+          // 0 * NaN would still poison P V, so that V tile is zeroed past kmax before use.
+          const bool fix = kv == 1 && kb <= kmax && kmax < kb + BN - 1 && ((kmax + 1) % 64) != 0;
+          uint64_t* land = fix ? &bars->v_fix : full;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(land, L::TILE);
+            const CUtensorMap* tm = kv ? tm_v : tm_k;
+            for (int half = 0; half < 2; ++half) {
+              const int pos0 = kb + 64 * half;
+              const int lp = pos0 / 64;
+              int64_t row = -1;  // outside the map: zero fill
+              if (pos0 <= kmax) {
+                int32_t page = -1;
+                if (lp < p.pt_stride) page = p.page_table[(int64_t)G.b * p.pt_stride + lp];
+                if (page < 0 || page >= p.pages) {
+                  record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+                } else {
+                  row = ((int64_t)p.full_layer * p.pages + page) * p.Hkv + G.g;
+                }
               }
+              for (int dh = 0; dh < D / 64; ++dh)
+                tma_load_3d(dst + dh * L::BLOCK + half * 64 * 128, tm, land, dh * 64, 0, (int)row);
             }
+          }
+          if (fix) {
+            __syncwarp();
+            if (!mbar_wait(&bars->v_fix, nfix & 1, p.err)) return;
+            ++nfix;
+            const int r0 = (int)(kmax - kb + 1);
+            for (int idx = lane; idx < (BN - r0) * (D / 8); idx += 32) {
+              const int r = r0 + idx / (D / 8);
+              const int c = idx % (D / 8);
+              *reinterpret_cast<uint4*>(dst + (c >> 3) * L::BLOCK + r * 128 + (c & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full);
+          }
+        } else if (j >= 0) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(full, L::TILE);
+            const CUtensorMap* tm = kv ? tm_v : tm_k;
             for (int dh = 0; dh < D / 64; ++dh)
-              tma_load_3d(dst + dh * L::BLOCK + half * 64 * 128, tm, land, dh * 64, 0, (int)row);
+              tma_load_4d(dst + dh * L::BLOCK, tm, full, dh * 64, G.g, (int)(BN * j), G.b);
           }
-        }
-        if (fix) {
-          __syncwarp();
-          if (!mbar_wait(&bars->v_fix, 0, p.err)) return;
-          const int r0 = (int)(kmax - kb + 1);
-          for (int idx = lane; idx < (BN - r0) * (D / 8); idx += 32) {
-            const int r = r0 + idx / (D / 8);
-            const int c = idx % (D / 8);
-            *reinterpret_cast<uint4*>(dst + (c >> 3) * L::BLOCK + r * 128 + (c & 7) * 16) = make_uint4(0, 0, 0, 0);
+        } else if (ring_fast) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(full, L::TILE);
+            const CUtensorMap* tm = kv ? tm_rv : tm_rk;
+            const int slot = (int)(kb % p.window);
+            int row = -1;  // outside the map: zero fill
+            if (seq >= 0 && seq < p.max_seqs)
+              row = (int)(((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + G.g);
+            else
+              record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+            for (int dh = 0; dh < D / 64; ++dh) tma_load_3d(dst + dh * L::BLOCK, tm, full, dh * 64, slot, row);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
+        } else {
+          ring_tile_cpasync<D>(p, G, kv ? p.ring_v : p.ring_k, dst, kb, lane);
           if (lane == 0) mbar_arrive(full);
         }
-      } else if (j >= 0) {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(full, L::TILE);
-          const CUtensorMap* tm = kv ? tm_v : tm_k;
-          for (int dh = 0; dh < D / 64; ++dh)
-            tma_load_4d(dst + dh * L::BLOCK, tm, full, dh * 64, G.g, (int)(BN * j), G.b);
-        }
-      } else if (ring_fast) {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(full, L::TILE);
-          const CUtensorMap* tm = kv ? tm_rv : tm_rk;
-          const int slot = (int)(kb % p.window);
-          int row = -1;  // outside the map: zero fill
-          if (seq >= 0 && seq < p.max_seqs)
-            row = (int)(((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + G.g);
-          else
-            record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
-          for (int dh = 0; dh < D / 64; ++dh) tma_load_3d(dst + dh * L::BLOCK, tm, full, dh * 64, slot, row);
-        }
-      } else {
-        ring_tile_cpasync<D>(p, G, kv ? p.ring_v : p.ring_k, dst, kb, lane);
-        if (lane == 0) mbar_arrive(full);
+        __syncwarp();
       }
-      __syncwarp();
     }
   }
 }
@@ -270,7 +303,7 @@ __device__ void producer(const Params& p, const Geo& G, uint8_t* smem, Bars* bar
 // ---------------------------------------------------------------- MMA issuer
 
 template <int D>
-__device__ void mma_issuer(const Params& p, const Geo& G, uint8_t* smem, Bars* bars, uint32_t tbase) {
+__device__ void mma_issuer(const Params& p, uint8_t* smem, Bars* bars, uint32_t tbase) {
   using L = Layout<D>;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
@@ -278,202 +311,262 @@ __device__ void mma_issuer(const Params& p, const Geo& G, uint8_t* smem, Bars* b
   const uint32_t k_base = smem_u32(smem + L::K_OFF);
   const uint32_t v_base = smem_u32(smem + L::V_OFF);
 
-  if (!mbar_wait(&bars->q_full, 0, p.err)) return;
-  tc_fence_after();
-
-  bool pend[NQT] = {false, false};
-  bool started[NQT] = {false, false};
-  uint32_t np[NQT] = {0, 0};
-  int prev_s = 0;
-  uint32_t prev_ph = 0;
-  int it = 0;
-
-  auto issue_pv = [&](int q, int s) {
-    const uint32_t d_tmem = tbase + L::O_COL0 + q * L::O_STRIDE;
-    const uint32_t a_tmem = tbase + q * 128;
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-      const uint64_t bdesc = smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, L::BLOCK, 1024);
-      umma_ts(d_tmem, a_tmem + kk * 8, bdesc, IDESC_PV, (started[q] || kk > 0) ? 1u : 0u);
-    }
-    started[q] = true;
-  };
-
-  for (int64_t j = G.jb; j <= G.je; ++j, ++it) {
-    const int s = it % NSTAGE;
-    const uint32_t ph = (it / NSTAGE) & 1;
-    if (!mbar_wait(&bars->k_full[s], ph, p.err)) return;
+  uint32_t np[NQT] = {0, 0};  // P tiles consumed per query tile (p_full phase)
+  int it = 0;                 // K/V tiles consumed (stage ring position)
+  uint32_t uq = 0;
+  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++uq) {
+    Geo G;
+    make_geo(p, unit, G);
+    if (!mbar_wait(&bars->q_full, uq & 1, p.err)) return;
     tc_fence_after();
-    bool v_ready = false;
-    for (int q = 0; q < NQT; ++q) {
-      if (pend[q]) {
-        if (!mbar_wait(&bars->p_full[q], np[q] & 1, p.err)) return;
-        ++np[q];
+
+    bool pend[NQT] = {false, false};
+    bool started[NQT] = {false, false};
+    int prev_s = 0;
+    uint32_t prev_ph = 0;
+    bool have_prev = false;
+
+    auto issue_pv = [&](int q, int s) {
+      const uint32_t d_tmem = tbase + L::O_COL0 + q * L::O_STRIDE;
+      const uint32_t a_tmem = tbase + q * 128;
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        const uint64_t bdesc = smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, L::BLOCK, 1024);
+        umma_ts(d_tmem, a_tmem + kk * 8, bdesc, IDESC_PV, (started[q] || kk > 0) ? 1u : 0u);
+      }
+      started[q] = true;
+    };
+    auto drain_q = [&](int q, bool& v_ready) -> bool {
+      if (!mbar_wait(&bars->p_full[q], np[q] & 1, p.err)) return false;
+      ++np[q];
+      tc_fence_after();
+      if (!v_ready) {
+        if (!mbar_wait(&bars->v_full[prev_s], prev_ph, p.err)) return false;
         tc_fence_after();
+        v_ready = true;
+      }
+      issue_pv(q, prev_s);
+      pend[q] = false;
+      return true;
+    };
+
+    for (int j = G.jb; j <= G.je; ++j, ++it) {
+      const int s = it % NSTAGE;
+      const uint32_t ph = (it / NSTAGE) & 1;
+      if (!mbar_wait(&bars->k_full[s], ph, p.err)) return;
+      tc_fence_after();
+      bool v_ready = false;
+      for (int q = 0; q < NQT; ++q) {
+        if (pend[q] && !drain_q(q, v_ready)) return;
+        if (needs(G, q, j)) {
+          const uint32_t d_tmem = tbase + q * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::BLOCK + (kk & 3) * 32;
+            const uint64_t adesc = smem_desc_sw128(q_base + q * L::TILE + off, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
+            umma_ss(d_tmem, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full[q]);
+          pend[q] = true;
+        }
+      }
+      umma_commit(&bars->k_empty[s]);
+      if (have_prev) {
         if (!v_ready) {
           if (!mbar_wait(&bars->v_full[prev_s], prev_ph, p.err)) return;
           tc_fence_after();
-          v_ready = true;
         }
-        issue_pv(q, prev_s);
-        pend[q] = false;
+        umma_commit(&bars->v_empty[prev_s]);
       }
-      if (needs(G, q, j)) {
-        const uint32_t d_tmem = tbase + q * 128;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::BLOCK + (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(q_base + q * L::TILE + off, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
-          umma_ss(d_tmem, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars->s_full[q]);
-        pend[q] = true;
-      }
+      prev_s = s;
+      prev_ph = ph;
+      have_prev = true;
     }
-    umma_commit(&bars->k_empty[s]);
-    if (it > 0) {
+    // every S MMA of the unit is issued: the Q buffers can be refilled once they complete
+    umma_commit(&bars->q_empty);
+    // drain the last tile's P V products and release its V stage
+    bool v_ready = false;
+    for (int q = 0; q < NQT; ++q)
+      if (pend[q] && !drain_q(q, v_ready)) return;
+    if (have_prev) {
       if (!v_ready) {
         if (!mbar_wait(&bars->v_full[prev_s], prev_ph, p.err)) return;
         tc_fence_after();
       }
       umma_commit(&bars->v_empty[prev_s]);
     }
-    prev_s = s;
-    prev_ph = ph;
+    for (int q = 0; q < NQT; ++q)
+      if (G.act[q]) umma_commit(&bars->o_full[q]);
   }
-  // drain the last tile's P V products
-  bool v_ready = false;
-  for (int q = 0; q < NQT; ++q) {
-    if (!pend[q]) continue;
-    if (!mbar_wait(&bars->p_full[q], np[q] & 1, p.err)) return;
-    ++np[q];
-    tc_fence_after();
-    if (!v_ready) {
-      if (!mbar_wait(&bars->v_full[prev_s], prev_ph, p.err)) return;
-      tc_fence_after();
-      v_ready = true;
-    }
-    issue_pv(q, prev_s);
-  }
-  for (int q = 0; q < NQT; ++q)
-    if (G.act[q]) umma_commit(&bars->o_full[q]);
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
 
-template <int D>
-__device__ void softmax_wg(const Params& p, const Geo& G, Bars* bars, uint32_t tbase, int q) {
+template <int D, int q>
+__device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase) {
   using L = Layout<D>;
-  if (!G.act[q]) return;
   const int wq = (threadIdx.x >> 5) & 3;
   const int lane = threadIdx.x & 31;
   const int r = wq * 32 + lane;
-  const int64_t i = G.i0[q] + r;
-  const int64_t lo_i = window_lo(p, i);
   const uint32_t trow = tbase + ((uint32_t)(wq * 32) << 16);
   const uint32_t s_col = q * 128;
   const uint32_t o_col = L::O_COL0 + q * L::O_STRIDE;
   const float sl2 = p.scale_log2;
+  uint32_t ns = 0;  // S tiles consumed (s_full phase)
+  uint32_t no = 0;  // units finished (o_full phase)
 
-  float m_used = -INFINITY;
-  float l = 0.f;
-  uint32_t n_done = 0;
+  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
+    Geo G;
+    make_geo(p, unit, G);
+    if (!G.act[q]) continue;
+    const int i = G.i0[q] + r;
+    const int lo_i = window_lo(p, i);
+    float m_used = -INFINITY;
+    float l = 0.f;
+    uint32_t n_done = 0;
 
-  for (int64_t j = G.jlo[q]; j <= G.jhi[q]; ++j) {
-    if (!mbar_wait(&bars->s_full[q], n_done & 1, p.err)) return;
-    tc_fence_after();
-    const int64_t kb = key_base(p, G, j);
-    const bool full_tile = mask_free(p, G, q, j);
-    // column range of this row inside the band
-    const int64_t c_lo = lo_i - kb;
-    const int64_t c_hi = i - kb;
-
-    float mx = -INFINITY;
+    for (int j = G.jlo[q]; j <= G.jhi[q]; ++j) {
+      if (!mbar_wait(&bars->s_full[q], ns & 1, p.err)) return;
+      ++ns;
+      tc_fence_after();
+      // columns of this row inside the band: [c_lo, c_hi] (edge tiles only)
+      const bool edge = !mask_free(p, G, q, j);
+      const int kb = key_base(p, G, j);
+      const int c_lo = lo_i - kb;
+      const int c_hi = i - kb;
+      // pass 1: row maximum, 64 scores at a time
+      float mx = -INFINITY;
 #pragma unroll
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-      uint32_t v[32];
-      tmem_ld32(trow + s_col + c0, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        float sv = __uint_as_float(v[k]);
-        if (!full_tile && (c0 + k < c_lo || c0 + k > c_hi)) sv = -INFINITY;
-        mx = fmaxf(mx, sv);
-      }
-    }
-    const float m_tile = mx * sl2;
-    float alpha = 1.f;
-    bool resc = false;
-    if (m_tile > m_used + kTau) {
-      if (m_used != -INFINITY) {
-        alpha = ex2_approx(m_used - m_tile);
-        resc = true;
-      }
-      l *= alpha;
-      m_used = m_tile;
-    }
-    if (__any_sync(0xffffffffu, resc) && n_done > 0) {
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + o_col + c0, v);
+      for (int h2 = 0; h2 < BN; h2 += 64) {
+        uint32_t va[32], vb[32];
+        tmem_ld32(trow + s_col + h2, va);
+        tmem_ld32(trow + s_col + h2 + 32, vb);
         tmem_wait_ld();
+        reg_fence32(va);
+        reg_fence32(vb);
+        if (edge) {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-        tmem_st32(trow + o_col + c0, v);
+          for (int k = 0; k < 32; ++k) {
+            if (h2 + k < c_lo || h2 + k > c_hi) va[k] = __float_as_uint(-INFINITY);
+            if (h2 + 32 + k < c_lo || h2 + 32 + k > c_hi) vb[k] = __float_as_uint(-INFINITY);
+          }
+        }
+        float m0 = mx, m1 = __uint_as_float(va[0]), m2 = __uint_as_float(vb[0]);
+#pragma unroll
+        for (int k = 1; k < 31; k += 2) {
+          m0 = fmax3(m0, __uint_as_float(va[k]), __uint_as_float(va[k + 1]));
+          m1 = fmax3(m1, __uint_as_float(vb[k]), __uint_as_float(vb[k + 1]));
+        }
+        m2 = fmax3(m2, __uint_as_float(va[31]), __uint_as_float(vb[31]));
+        mx = fmax3(m0, m1, m2);
       }
-      tmem_wait_st();
-    }
-    const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+      const float m_tile = mx * sl2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_tile > m_used + kTau) {
+        if (m_used != -INFINITY) {
+          alpha = ex2_approx(m_used - m_tile);
+          resc = true;
+        }
+        l *= alpha;
+        m_used = m_tile;
+      }
+      if (__any_sync(0xffffffffu, resc) && n_done > 0) {
 #pragma unroll
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-      uint32_t v[32];
-      tmem_ld32(trow + s_col + c0, v);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(trow + o_col + c0, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(trow + o_col + c0, o);
+        }
+        tmem_wait_st();
+      }
+      // pass 2: P = 2^(s * scale * log2 e - m), 32 columns at a time, the next chunk's TMEM
+      // load in flight while this one is exponentiated, packed and stored over S.
+      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+      const uint64_t scale2 = f2_pack(sl2, sl2);
+      const uint64_t neg2 = f2_pack(-moff, -moff);
+      uint64_t acc[4] = {0, 0, 0, 0};
+      uint32_t buf[2][32];
+      tmem_ld32(trow + s_col, buf[0]);
       tmem_wait_ld();
+      reg_fence32(buf[0]);
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t(&cur)[32] = buf[c & 1];
+        if (c + 1 < BN / 32) tmem_ld32(trow + s_col + 32 * (c + 1), buf[(c + 1) & 1]);
+        const int c0 = 32 * c;
+        if (edge) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (c0 + k < c_lo || c0 + k > c_hi) cur[k] = __float_as_uint(-INFINITY);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const int pair = (c0 + k) >> 1;
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(cur[k]), __uint_as_float(cur[k + 1])), scale2, neg2);
+          uint64_t e;
+          if ((pair % kPolyEvery) == kPolyEvery - 1) {
+            e = exp2_poly_x2(x);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc[pair & 3] = f2_add(acc[pair & 3], e);
+          float e0, e1;
+          f2_unpack(e, e0, e1);
+          pk[k >> 1] = pack_bf16x2(e0, e1);
+        }
+        tmem_st16(trow + s_col + (c0 >> 1), pk);
+        if (c + 1 < BN / 32) {
+          tmem_wait_ld();
+          reg_fence32(buf[(c + 1) & 1]);
+        }
+      }
+      float a0, a1, b0, b1, c0_, c1_, d0, d1;
+      f2_unpack(acc[0], a0, a1);
+      f2_unpack(acc[1], b0, b1);
+      f2_unpack(acc[2], c0_, c1_);
+      f2_unpack(acc[3], d0, d1);
+      l += ((a0 + a1) + (b0 + b1)) + ((c0_ + c1_) + (d0 + d1));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[q]);
+      ++n_done;
+    }
+
+    if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
+    ++no;
+    tc_fence_after();
+    const int64_t row = (int64_t)G.t[q] * BM + r;
+    const bool valid = row < p.n_q;
+    const float inv = 1.f / l;
+    uint16_t* out = p.o + (((int64_t)G.b * p.n_q + row) * p.Hq + G.h) * D;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld32(trow + o_col + c0, o);
+      tmem_wait_ld();
+      reg_fence32(o);
       uint32_t pk[16];
 #pragma unroll
-      for (int k = 0; k < 32; k += 2) {
-        float s0 = __uint_as_float(v[k]);
-        float s1 = __uint_as_float(v[k + 1]);
-        if (!full_tile) {
-          if (c0 + k < c_lo || c0 + k > c_hi) s0 = -INFINITY;
-          if (c0 + k + 1 < c_lo || c0 + k + 1 > c_hi) s1 = -INFINITY;
-        }
-        const float p0 = ex2_approx(fmaf(s0, sl2, -moff));
-        const float p1 = ex2_approx(fmaf(s1, sl2, -moff));
-        l += p0 + p1;
-        pk[k >> 1] = pack_bf16x2(p0, p1);
+      for (int k = 0; k < 32; k += 2)
+        pk[k >> 1] = pack_bf16x2(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv);
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + c0);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
       }
-      tmem_st16(trow + s_col + (c0 >> 1), pk);
     }
-    tmem_wait_st();
+    // O of this query tile has been read: the next unit's first P V may overwrite it
+    // (ordered by this warpgroup's next p_full arrival).
     tc_fence_before();
-    mbar_arrive(&bars->p_full[q]);
-    ++n_done;
-  }
-
-  if (n_done == 0) return;
-  if (!mbar_wait(&bars->o_full[q], 0, p.err)) return;
-  tc_fence_after();
-  const int64_t row = (int64_t)G.t[q] * BM + r;
-  const bool valid = row < p.n_q;
-  const float inv = 1.f / l;
-  uint16_t* out = p.o + (((int64_t)G.b * p.n_q + row) * p.Hq + G.h) * D;
-#pragma unroll
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    uint32_t v[32];
-    tmem_ld32(trow + o_col + c0, v);
-    tmem_wait_ld();
-    uint32_t pk[16];
-#pragma unroll
-    for (int k = 0; k < 32; k += 2)
-      pk[k >> 1] = pack_bf16x2(__uint_as_float(v[k]) * inv, __uint_as_float(v[k + 1]) * inv);
-    if (valid) {
-      uint4* dst = reinterpret_cast<uint4*>(out + c0);
-#pragma unroll
-      for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-    }
   }
 }
 
@@ -490,11 +583,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (read_error(p.err) != 0) return;  // a pending device error: skip the work
 
-  Geo G;
-  make_geo(p, G);
-
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
@@ -509,12 +600,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars->v_fix, 1);
     fence_barrier_init();
   }
-  if (warp == 0 && (threadIdx.x & 31) == 0) {
+  if (warp == PRODUCER_WARP && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -523,18 +614,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
 
-  if (warp == 0) {
-    producer<D>(p, G, smem, bars, &tm_q, &tm_k, &tm_v, &tm_rk, &tm_rv);
-  } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) mma_issuer<D>(p, G, smem, bars, tbase);
+  if (warp < 4) {
+    softmax_wg<D, 0>(p, bars, tbase);
+  } else if (warp < 8) {
+    softmax_wg<D, 1>(p, bars, tbase);
+  } else if (warp == PRODUCER_WARP) {
+    producer<D>(p, smem, bars, &tm_q, &tm_k, &tm_v, &tm_rk, &tm_rv);
+  } else {
+    if ((threadIdx.x & 31) == 0) mma_issuer<D>(p, smem, bars, tbase);
     __syncwarp();
-  } else if (warp >= 4) {
-    softmax_wg<D>(p, G, bars, tbase, (warp - 4) >> 2);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -568,13 +661,22 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
   p.pages = D.pages_per_full_layer;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)Lc.d));
   p.n_pairs = (int)((Lc.n_q + BM * NQT - 1) / (BM * NQT));
+  p.max_start = 0x7fffffffLL - Lc.n_q - 2 * BN;
   p.err = pool->err;
   if (Lc.n_q == 0 || Lc.B == 0) return HSWA_OK;
+  const int64_t units = (int64_t)p.n_pairs * Lc.B * Lc.Hq;
+  if (units > 0x7fffffff) {
+    set_error("prefill: too many work units");
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  p.n_units = (int)units;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.n_units < sms ? p.n_units : sms;
 
-  const dim3 grid(Lc.Hq, p.n_pairs, Lc.B);
   const CUtensorMap& rk = pool->ring_tma ? pool->tm_ring_k : Lc.tm_k;
   const CUtensorMap& rv = pool->ring_tma ? pool->tm_ring_v : Lc.tm_v;
-  cudaError_t e;
   if (Lc.d == 128) {
     const int smem = Layout<128>::BYTES + 1024;
     cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -584,7 +686,7 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
     cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     prefill_kernel<64><<<grid, NTHREADS, smem, stream>>>(p, Lc.tm_q, Lc.tm_k, Lc.tm_v, rk, rv);
   }
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("prefill: launch failed: %s", cudaGetErrorString(e));
     return HSWA_ERR_CUDA;
