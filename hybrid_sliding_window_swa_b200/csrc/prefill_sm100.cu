@@ -19,6 +19,8 @@
 //               in the exp2 domain with lazy O rescaling, exponentials split between
 //               the MUFU unit and an FMA-pipe polynomial, P written back over S as
 //               packed bf16, and the epilogue (O / l -> bf16 -> global).
+//   warps 8-11  a third warpgroup that gives its registers to the softmax warpgroups
+//               (setmaxnreg: 2 x 128 x 208 + 128 x 88 = the 384 x 168 the CTA launches with):
 //   warp 8      producer: Q of each unit, then K/V tiles into a 2-stage ring of
 //               shared-memory buffers (TMA for chunk rows, aligned ring tiles and
 //               pages; cp.async for rolling-buffer rows that are not 128-aligned).
@@ -41,7 +43,7 @@ constexpr int BM = 128;     // query rows per tile
 constexpr int BN = 128;     // keys per tile
 constexpr int NQT = 2;      // query tiles per unit
 constexpr int NSTAGE = 2;   // K/V pipeline depth
-constexpr int NWARPS = 10;
+constexpr int NWARPS = 12;         // 3 warpgroups: registers are granted per warpgroup
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
@@ -403,8 +405,8 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
 
 // ---------------------------------------------------------------- softmax + epilogue
 
-template <int D, int q>
-__device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase) {
+template <int D>
+__device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase, const int q) {
   using L = Layout<D>;
   const int wq = (threadIdx.x >> 5) & 3;
   const int lane = threadIdx.x & 31;
@@ -419,20 +421,28 @@ __device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase) {
   for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
     Geo G;
     make_geo(p, unit, G);
-    if (!G.act[q]) continue;
-    const int i = G.i0[q] + r;
+    // this warpgroup's query tile, as scalars (one code path for both warpgroups)
+    const bool act = q ? G.act[1] : G.act[0];
+    if (!act) continue;
+    const int qi0 = q ? G.i0[1] : G.i0[0];
+    const int qi1 = q ? G.i1[1] : G.i1[0];
+    const int qjlo = q ? G.jlo[1] : G.jlo[0];
+    const int qjhi = q ? G.jhi[1] : G.jhi[0];
+    const int qt = q ? G.t[1] : G.t[0];
+    const int lo_last = window_lo(p, qi1);
+    const int i = qi0 + r;
     const int lo_i = window_lo(p, i);
     float m_used = -INFINITY;
     float l = 0.f;
     uint32_t n_done = 0;
 
-    for (int j = G.jlo[q]; j <= G.jhi[q]; ++j) {
+    for (int j = qjlo; j <= qjhi; ++j) {
       if (!mbar_wait(&bars->s_full[q], ns & 1, p.err)) return;
       ++ns;
       tc_fence_after();
       // columns of this row inside the band: [c_lo, c_hi] (edge tiles only)
-      const bool edge = !mask_free(p, G, q, j);
       const int kb = key_base(p, G, j);
+      const bool edge = !(kb + BN - 1 <= qi0 && kb >= lo_last);
       const int c_lo = lo_i - kb;
       const int c_hi = i - kb;
       // pass 1: row maximum, 64 scores at a time
@@ -544,7 +554,7 @@ __device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase) {
     if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
     ++no;
     tc_fence_after();
-    const int64_t row = (int64_t)G.t[q] * BM + r;
+    const int64_t row = (int64_t)qt * BM + r;
     const bool valid = row < p.n_q;
     const float inv = 1.f / l;
     uint16_t* out = p.o + (((int64_t)G.b * p.n_q + row) * p.Hq + G.h) * D;
@@ -614,15 +624,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tbase = bars->tmem_base;
 
-  if (warp < 4) {
-    softmax_wg<D, 0>(p, bars, tbase);
-  } else if (warp < 8) {
-    softmax_wg<D, 1>(p, bars, tbase);
-  } else if (warp == PRODUCER_WARP) {
-    producer<D>(p, smem, bars, &tm_q, &tm_k, &tm_v, &tm_rk, &tm_rv);
+  if (warp < 8) {
+    // two softmax warpgroups take the registers the third one gives back
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    softmax_wg<D>(p, bars, tbase, warp >> 2);
   } else {
-    if ((threadIdx.x & 31) == 0) mma_issuer<D>(p, smem, bars, tbase);
-    __syncwarp();
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+    if (warp == PRODUCER_WARP) {
+      producer<D>(p, smem, bars, &tm_q, &tm_k, &tm_v, &tm_rk, &tm_rv);
+    } else if (warp == MMA_WARP) {
+      if ((threadIdx.x & 31) == 0) mma_issuer<D>(p, smem, bars, tbase);
+      __syncwarp();
+    }
   }
 
   tc_fence_before();
