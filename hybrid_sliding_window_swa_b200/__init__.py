@@ -54,7 +54,7 @@ def load_library(path: str | None = None):
     global _lib
     if _lib is not None:
         return _lib
-    path = path or LIB_PATH
+    path = path or os.environ.get("HSWA_LIBRARY") or LIB_PATH
     if not os.path.exists(path):
         raise ImportError(f"libhswa.so not found at {path}; build it with "
                           f"`python -m hybrid_sliding_window_swa_b200._build`")

@@ -29,7 +29,12 @@ def _stale(out: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, defines=(),
+          lib_path: str | None = None, build_dir: str | None = None) -> str:
+    """Compile the library; `defines` (e.g. ["HSWA_POLY_PER8=3"]) select tuning parameters and
+    `lib_path`/`build_dir` place a variant build elsewhere."""
+    LIB = lib_path or globals()["LIB"]
+    BUILD_DIR = build_dir or globals()["BUILD_DIR"]
     os.makedirs(BUILD_DIR, exist_ok=True)
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(HERE, "..", "include", "hswa.h")]
     objs = []
@@ -39,7 +44,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
         op = os.path.join(BUILD_DIR, src.replace(".cu", ".o"))
         objs.append(op)
         if force or _stale(op, [sp] + hdrs):
-            cmd = [NVCC, *FLAGS, "-c", sp, "-o", op]
+            cmd = [NVCC, *FLAGS, *[f"-D{d}" for d in defines], "-c", sp, "-o", op]
             if ptxas_verbose:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)

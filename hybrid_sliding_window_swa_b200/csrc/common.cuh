@@ -231,6 +231,18 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
+template <int B, int N>
+__device__ __forceinline__ void reg_fence_into(uint32_t (&r)[N]) {
+  static_assert(B + 32 <= N, "range");
+  asm volatile(""
+               : "+r"(r[B + 0]), "+r"(r[B + 1]), "+r"(r[B + 2]), "+r"(r[B + 3]), "+r"(r[B + 4]), "+r"(r[B + 5]),
+                 "+r"(r[B + 6]), "+r"(r[B + 7]), "+r"(r[B + 8]), "+r"(r[B + 9]), "+r"(r[B + 10]), "+r"(r[B + 11]),
+                 "+r"(r[B + 12]), "+r"(r[B + 13]), "+r"(r[B + 14]), "+r"(r[B + 15]), "+r"(r[B + 16]),
+                 "+r"(r[B + 17]), "+r"(r[B + 18]), "+r"(r[B + 19]), "+r"(r[B + 20]), "+r"(r[B + 21]),
+                 "+r"(r[B + 22]), "+r"(r[B + 23]), "+r"(r[B + 24]), "+r"(r[B + 25]), "+r"(r[B + 26]),
+                 "+r"(r[B + 27]), "+r"(r[B + 28]), "+r"(r[B + 29]), "+r"(r[B + 30]), "+r"(r[B + 31]));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "

@@ -20,7 +20,7 @@
 //               the MUFU unit and an FMA-pipe polynomial, P written back over S as
 //               packed bf16, and the epilogue (O / l -> bf16 -> global).
 //   warps 8-11  a third warpgroup that gives its registers to the softmax warpgroups
-//               (setmaxnreg: 2 x 128 x 208 + 128 x 88 = the 384 x 168 the CTA launches with):
+//               (setmaxnreg, by default 2 x 128 x 208 + 128 x 88 = the 384 x 168 the CTA launches with):
 //   warp 8      producer: Q of each unit, then K/V tiles into a 2-stage ring of
 //               shared-memory buffers (TMA for chunk rows, aligned ring tiles and
 //               pages; cp.async for rolling-buffer rows that are not 128-aligned).
@@ -48,7 +48,29 @@ constexpr int NTHREADS = NWARPS * 32;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <= 2^8
-constexpr int kPolyEvery = 4; // one pair in kPolyEvery takes the FMA-pipe exponential
+
+// Tuning parameters (compile-time):
+//  HSWA_POLY_PER8           pairs of scores in every 8 whose exponential runs on the FMA pipe
+//  HSWA_SOFTMAX_SINGLE_PASS 1: keep all 128 scores of a row in registers (one TMEM read);
+//                           0: read S twice (row maximum, then exponentials), fewer registers
+//  HSWA_SOFTMAX_REGS / HSWA_PRODUCER_REGS  setmaxnreg split (2 * 128 * a + 128 * b <= 384 * 168)
+#ifndef HSWA_POLY_PER8
+#define HSWA_POLY_PER8 2
+#endif
+#ifndef HSWA_SOFTMAX_SINGLE_PASS
+#define HSWA_SOFTMAX_SINGLE_PASS 0
+#endif
+#ifndef HSWA_SOFTMAX_REGS
+#define HSWA_SOFTMAX_REGS 208
+#endif
+#ifndef HSWA_PRODUCER_REGS
+#define HSWA_PRODUCER_REGS 88
+#endif
+static_assert(2 * 128 * HSWA_SOFTMAX_REGS + 128 * HSWA_PRODUCER_REGS <= 384 * 168, "register split");
+#define HSWA_STR2(x) #x
+#define HSWA_STR(x) HSWA_STR2(x)
+
+__device__ __forceinline__ constexpr bool use_poly(int pair) { return (pair & 7) >= 8 - HSWA_POLY_PER8; }
 
 struct Params {
   int B, n_q, Hq, Hkv, G;
@@ -445,6 +467,87 @@ __device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase, const in
       const bool edge = !(kb + BN - 1 <= qi0 && kb >= lo_last);
       const int c_lo = lo_i - kb;
       const int c_hi = i - kb;
+#if HSWA_SOFTMAX_SINGLE_PASS
+      // all 128 scores of the row: four TMEM loads, one wait
+      uint32_t v[128];
+      tmem_ld32_into<0>(trow + s_col + 0, v);
+      tmem_ld32_into<32>(trow + s_col + 32, v);
+      tmem_ld32_into<64>(trow + s_col + 64, v);
+      tmem_ld32_into<96>(trow + s_col + 96, v);
+      tmem_wait_ld();
+      reg_fence_into<0>(v);
+      reg_fence_into<32>(v);
+      reg_fence_into<64>(v);
+      reg_fence_into<96>(v);
+      if (edge) {
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k < c_lo || k > c_hi) v[k] = __float_as_uint(-INFINITY);
+      }
+      float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
+      float m2 = __uint_as_float(v[2]), m3 = __uint_as_float(v[3]);
+#pragma unroll
+      for (int k = 4; k < 124; k += 8) {
+        m0 = fmax3(m0, __uint_as_float(v[k + 0]), __uint_as_float(v[k + 1]));
+        m1 = fmax3(m1, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+        m2 = fmax3(m2, __uint_as_float(v[k + 4]), __uint_as_float(v[k + 5]));
+        m3 = fmax3(m3, __uint_as_float(v[k + 6]), __uint_as_float(v[k + 7]));
+      }
+      m0 = fmax3(m0, __uint_as_float(v[124]), __uint_as_float(v[125]));
+      m1 = fmax3(m1, __uint_as_float(v[126]), __uint_as_float(v[127]));
+      const float mx = fmaxf(fmax3(m0, m1, m2), m3);
+      const float m_tile = mx * sl2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_tile > m_used + kTau) {
+        if (m_used != -INFINITY) {
+          alpha = ex2_approx(m_used - m_tile);
+          resc = true;
+        }
+        l *= alpha;
+        m_used = m_tile;
+      }
+      if (__any_sync(0xffffffffu, resc) && n_done > 0) {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(trow + o_col + c0, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(trow + o_col + c0, o);
+        }
+        tmem_wait_st();
+      }
+      // P = 2^(s * scale * log2 e - m) in place, packed to bf16 and stored over S
+      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+      const uint64_t scale2 = f2_pack(sl2, sl2);
+      const uint64_t neg2 = f2_pack(-moff, -moff);
+      uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const int pair = (c0 + k) >> 1;
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(v[c0 + k]), __uint_as_float(v[c0 + k + 1])), scale2, neg2);
+          uint64_t e;
+          if (use_poly(pair)) {
+            e = exp2_poly_x2(x);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc[pair & 3] = f2_add(acc[pair & 3], e);
+          float e0, e1;
+          f2_unpack(e, e0, e1);
+          pk[k >> 1] = pack_bf16x2(e0, e1);
+        }
+        tmem_st16(trow + s_col + (c0 >> 1), pk);
+      }
+#else
       // pass 1: row maximum, 64 scores at a time
       float mx = -INFINITY;
 #pragma unroll
@@ -521,7 +624,7 @@ __device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase, const in
           const int pair = (c0 + k) >> 1;
           const uint64_t x = f2_fma(f2_pack(__uint_as_float(cur[k]), __uint_as_float(cur[k + 1])), scale2, neg2);
           uint64_t e;
-          if ((pair % kPolyEvery) == kPolyEvery - 1) {
+          if (use_poly(pair)) {
             e = exp2_poly_x2(x);
           } else {
             float x0, x1;
@@ -539,6 +642,7 @@ __device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase, const in
           reg_fence32(buf[(c + 1) & 1]);
         }
       }
+#endif
       float a0, a1, b0, b1, c0_, c1_, d0, d1;
       f2_unpack(acc[0], a0, a1);
       f2_unpack(acc[1], b0, b1);
@@ -626,10 +730,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp < 8) {
     // two softmax warpgroups take the registers the third one gives back
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 " HSWA_STR(HSWA_SOFTMAX_REGS) ";" ::: "memory");
     softmax_wg<D>(p, bars, tbase, warp >> 2);
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 " HSWA_STR(HSWA_PRODUCER_REGS) ";" ::: "memory");
     if (warp == PRODUCER_WARP) {
       producer<D>(p, smem, bars, &tm_q, &tm_k, &tm_v, &tm_rk, &tm_rv);
     } else if (warp == MMA_WARP) {
