@@ -20,7 +20,7 @@
 //               the MUFU unit and an FMA-pipe polynomial, P written back over S as
 //               packed bf16, and the epilogue (O / l -> bf16 -> global).
 //   warps 8-11  a third warpgroup that gives its registers to the softmax warpgroups
-//               (setmaxnreg, by default 2 x 128 x 208 + 128 x 88 = the 384 x 168 the CTA launches with):
+//               (setmaxnreg, by default 2 x 128 x 216 + 128 x 72 = the 384 x 168 the CTA launches with):
 //   warp 8      producer: Q of each unit, then K/V tiles into a 2-stage ring of
 //               shared-memory buffers (TMA for chunk rows, aligned ring tiles and
 //               pages; cp.async for rolling-buffer rows that are not 128-aligned).
@@ -58,13 +58,13 @@ constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <=
 #define HSWA_POLY_PER8 2
 #endif
 #ifndef HSWA_SOFTMAX_SINGLE_PASS
-#define HSWA_SOFTMAX_SINGLE_PASS 0
+#define HSWA_SOFTMAX_SINGLE_PASS 1
 #endif
 #ifndef HSWA_SOFTMAX_REGS
-#define HSWA_SOFTMAX_REGS 208
+#define HSWA_SOFTMAX_REGS 216
 #endif
 #ifndef HSWA_PRODUCER_REGS
-#define HSWA_PRODUCER_REGS 88
+#define HSWA_PRODUCER_REGS 72
 #endif
 static_assert(2 * 128 * HSWA_SOFTMAX_REGS + 128 * HSWA_PRODUCER_REGS <= 384 * 168, "register split");
 #define HSWA_STR2(x) #x
