@@ -180,7 +180,8 @@ template <int D, int MT>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
   using SM = DecSmem<D, MT>;
   constexpr int ROWS = SM::ROWS;
-  constexpr int CH = D / 8;  // 16-byte chunks per row
+  constexpr int CH = D / 8;              // 16-byte chunks per row
+  constexpr int ROWS_PER_PASS = 512 / (D * 2);  // rows one warp-wide 16-byte copy covers
   extern __shared__ __align__(128) uint8_t smem[];
   float* m_w = reinterpret_cast<float*>(smem + SM::MISC_OFF);   // [4][ROWS]
   float* l_w = m_w + 4 * ROWS;                                  // [4][ROWS]
@@ -194,6 +195,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
   const int* prefix = reinterpret_cast<const int*>(p.ws + sizeof(WsHeader));
 
   if (read_error(p.err) != 0) return;
+
+  // this thread's fixed place in a 64-row block copy: row (within a pass), 16-byte chunk
+  const int cp_row = tid / CH;                  // 0 .. 128/CH - 1
+  const int cp_chunk = tid % CH;
+  constexpr int CP_ROWS = DEC_THREADS / CH;     // rows covered by the CTA per copy instruction
+  static_assert(KB % CP_ROWS == 0, "block rows");
 
   for (;;) {
     if (tid == 0) *item_slot = atomicAdd(&hdr->counter, 1);
@@ -213,22 +220,28 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     const int c = sc - prefix[s];
     const int nsp = prefix[s + 1] - prefix[s];
     const bool last = c == nsp - 1;
-    const int64_t L = safe_len(p, s);
-    const int64_t klo = dec_klo(p, L);
-    const int64_t a = klo + (int64_t)c * SPLIT;
-    const int64_t b = (a + SPLIT < L) ? a + SPLIT : L;
-    const int n_cached_blk = (int)((b - a + KB - 1) / KB);
+    const int L = (int)safe_len(p, s);
+    const int klo = (int)dec_klo(p, L);
+    const int a = klo + c * SPLIT;
+    const int b = (a + SPLIT < L) ? a + SPLIT : L;
+    const int n_cached_blk = (b - a + KB - 1) / KB;
     const int n_blk = n_cached_blk + (last ? 1 : 0);
-    int64_t ring_row = 0;
+    // source rows of this (sequence, KV head)
+    const uint16_t* ring_k = nullptr;
+    const uint16_t* ring_v = nullptr;
+    bool src_ok = true;
     if (p.window > 0) {
       const int seq = p.seq_ids[s];
       if (seq < 0 || seq >= p.max_seqs) {
         record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
-        ring_row = -1;
+        src_ok = false;
       } else {
-        ring_row = (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + g) * p.window;
+        const int64_t row0 = (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + g) * p.window;
+        ring_k = p.src_k + row0 * D;
+        ring_v = p.src_v + row0 * D;
       }
     }
+    const int32_t* pt_row = p.page_table ? p.page_table + (int64_t)s * p.pt_stride : nullptr;
 
     // ---- stage Q rows (row = t * G + hh) into shared memory, zero rows >= R
     for (int idx = tid; idx < ROWS * CH; idx += DEC_THREADS) {
@@ -242,42 +255,58 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, ch)) = val;
     }
 
-    // ---- block loader: block kb2 of this item into stage st
+    // ---- block loader: block kb2 of this item into stage st. Each copy instruction of the CTA
+    // moves CP_ROWS whole rows (contiguous in HBM within a page or a ring run).
     auto load_block = [&](int kb2, int st) {
-      for (int idx = tid; idx < KB * CH; idx += DEC_THREADS) {
-        const int r = idx / CH, ch = idx % CH;
-        const uint16_t* sk = p.src_k;  // any valid address for zero-fill
-        const uint16_t* sv = p.src_v;
-        uint32_t bytes = 0;
-        if (kb2 < n_cached_blk) {
-          const int64_t pos = a + (int64_t)kb2 * KB + r;
-          if (pos < b) {
-            int64_t row = -1;
-            if (p.window > 0) {
-              if (ring_row >= 0) row = ring_row + pos % p.window;
-            } else {
-              const int64_t lp = pos / 64;
-              const int32_t page = lp < p.pt_stride ? p.page_table[(int64_t)s * p.pt_stride + lp] : -1;
-              if (page < 0 || page >= p.pages) {
-                record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
-              } else {
-                row = (((int64_t)p.full_layer * p.pages + page) * p.Hkv + g) * 64 + pos % 64;
-              }
-            }
-            if (row >= 0) {
-              sk = p.src_k + row * D + ch * 8;
-              sv = p.src_v + row * D + ch * 8;
-              bytes = 16;
-            }
+      const uint32_t kdst = s_base + SM::K_OFF + st * SM::TILE;
+      const uint32_t vdst = s_base + SM::V_OFF + st * SM::TILE;
+      if (kb2 < n_cached_blk) {
+        const int pos0 = a + kb2 * KB;
+        const int nvalid = b - pos0;  // rows of this block that exist (>= 1)
+        if (p.window > 0) {
+          int slot0 = pos0 % p.window;
+#pragma unroll
+          for (int rr = 0; rr < KB; rr += CP_ROWS) {
+            const int r = rr + cp_row;
+            int slot = slot0 + r;
+            if (slot >= p.window) slot = (p.window >= KB) ? slot - p.window : slot % p.window;
+            const bool ok = src_ok && r < nvalid;
+            const size_t off = ok ? (size_t)slot * D + cp_chunk * 8 : 0;
+            const uint16_t* sk = ok ? ring_k + off : p.src_k;
+            const uint16_t* sv = ok ? ring_v + off : p.src_v;
+            cp_async_16(kdst + sw_off<D>(r, cp_chunk), sk, ok ? 16u : 0u);
+            cp_async_16(vdst + sw_off<D>(r, cp_chunk), sv, ok ? 16u : 0u);
           }
-        } else if (r < p.n_qt) {
-          const int64_t row = ((int64_t)s * p.n_qt + r) * p.Hkv + g;
-          sk = p.k_new + row * D + ch * 8;
-          sv = p.v_new + row * D + ch * 8;
-          bytes = 16;
+        } else {
+          // a block is exactly one 64-token page (splits start at multiples of 64)
+          const int lp = pos0 / 64;
+          int32_t page = lp < p.pt_stride ? pt_row[lp] : -1;
+          bool ok_page = page >= 0 && page < p.pages;
+          if (!ok_page && tid == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+          const int64_t prow = ok_page ? (((int64_t)p.full_layer * p.pages + page) * p.Hkv + g) * 64 : 0;
+          const uint16_t* kbase = p.src_k + prow * D;
+          const uint16_t* vbase = p.src_v + prow * D;
+#pragma unroll
+          for (int rr = 0; rr < KB; rr += CP_ROWS) {
+            const int r = rr + cp_row;
+            const bool ok = ok_page && r < nvalid;
+            const int off = ok ? r * D + cp_chunk * 8 : 0;
+            cp_async_16(kdst + sw_off<D>(r, cp_chunk), ok ? kbase + off : p.src_k, ok ? 16u : 0u);
+            cp_async_16(vdst + sw_off<D>(r, cp_chunk), ok ? vbase + off : p.src_v, ok ? 16u : 0u);
+          }
         }
-        cp_async_16(s_base + SM::K_OFF + st * SM::TILE + sw_off<D>(r, ch), sk, bytes);
-        cp_async_16(s_base + SM::V_OFF + st * SM::TILE + sw_off<D>(r, ch), sv, bytes);
+      } else {
+        // the new tokens: rows 0 .. n_qt-1 of k_new / v_new, zeros after
+#pragma unroll
+        for (int rr = 0; rr < KB; rr += CP_ROWS) {
+          const int r = rr + cp_row;
+          const bool ok = r < p.n_qt;
+          const int64_t row = ((int64_t)s * p.n_qt + (ok ? r : 0)) * p.Hkv + g;
+          const uint16_t* sk = p.k_new + row * D + cp_chunk * 8;
+          const uint16_t* sv = p.v_new + row * D + cp_chunk * 8;
+          cp_async_16(kdst + sw_off<D>(r, cp_chunk), sk, ok ? 16u : 0u);
+          cp_async_16(vdst + sw_off<D>(r, cp_chunk), sv, ok ? 16u : 0u);
+        }
       }
     };
 
@@ -290,38 +319,37 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     // per-thread row state: rows (mt*16 + lane/4) and (+8)
     float o_acc[MT][D / 8][4];
     float m_r[MT][2], l_r[MT][2];
+    int row_pos[MT][2], row_lo[MT][2];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      m_r[mt][0] = m_r[mt][1] = -INFINITY;
-      l_r[mt][0] = l_r[mt][1] = 0.f;
-#pragma unroll
-      for (int nd = 0; nd < D / 8; ++nd) o_acc[mt][nd][0] = o_acc[mt][nd][1] = o_acc[mt][nd][2] = o_acc[mt][nd][3] = 0.f;
-    }
-    // per-row query token t and window start, for the two rows of each M tile
-    int64_t row_pos[MT][2], row_lo[MT][2];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
+        m_r[mt][hf] = -INFINITY;
+        l_r[mt][hf] = 0.f;
         const int r = mt * 16 + (lane >> 2) + hf * 8;
         const int t = r < p.R ? r / p.G : 0;
         row_pos[mt][hf] = L + t;
-        int64_t lo2 = 0;
+        int lo2 = 0;
         if (p.window > 0) {
           lo2 = L + t - p.window + 1;
           if (lo2 < 0) lo2 = 0;
         }
-        row_lo[mt][hf] = r < p.R ? lo2 : INT64_MAX;  // padding rows see nothing
+        row_lo[mt][hf] = r < p.R ? lo2 : 0x7fffffff;  // padding rows see nothing
       }
+#pragma unroll
+      for (int nd = 0; nd < D / 8; ++nd) o_acc[mt][nd][0] = o_acc[mt][nd][1] = o_acc[mt][nd][2] = o_acc[mt][nd][3] = 0.f;
+    }
+    // largest window start over the real rows: cached keys at or above it need no mask
+    const int lo_max = p.window > 0 ? (L + p.n_qt - 1 - p.window + 1 > 0 ? L + p.n_qt - p.window : 0) : 0;
 
     for (int kb2 = 0; kb2 < n_blk; ++kb2) {
+      asm volatile("cp.async.wait_group %0;" ::"n"(NST - 2) : "memory");
+      __syncthreads();  // block kb2 is visible; every warp is done with block kb2 - 1
       {
         const int nxt = kb2 + NST - 1;
         if (nxt < n_blk) load_block(nxt, nxt % NST);
         asm volatile("cp.async.commit_group;" ::: "memory");
       }
-      asm volatile("cp.async.wait_group %0;" ::"n"(NST - 1) : "memory");
-      __syncthreads();
       const int st = kb2 % NST;
       const uint32_t kt = s_base + SM::K_OFF + st * SM::TILE;
       const uint32_t vt = s_base + SM::V_OFF + st * SM::TILE;
@@ -352,10 +380,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           mma_bf16(sacc[mt][1], a0, a1, a2, a3, b2, b3);
         }
       }
-      // mask + online softmax (exp2 domain)
-      int64_t kpos_base;
-      bool is_new = kb2 >= n_cached_blk;
-      kpos_base = is_new ? L : a + (int64_t)kb2 * KB;
+      // mask (edge blocks only) + online softmax in the exp2 domain with lazy rescaling
+      const bool is_new = kb2 >= n_cached_blk;
+      const int kpos_base = is_new ? L : a + kb2 * KB;
+      const bool need_mask = is_new || kpos_base + KB > b || kpos_base < lo_max;
       uint32_t pa[MT][4];
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -366,34 +394,35 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int kcol = key0 + nt * 8 + (lane & 3) * 2 + e;
-              const int64_t pos = kpos_base + kcol;
-              bool ok;
-              if (is_new) ok = kcol < p.n_qt && pos <= row_pos[mt][hf] && pos >= row_lo[mt][hf];
-              else ok = pos < b && pos >= row_lo[mt][hf];
-              const float sv = sacc[mt][nt][hf * 2 + e];
-              v[nt * 2 + e] = ok ? sv * p.scale_log2 : -INFINITY;
+              const float sv = sacc[mt][nt][hf * 2 + e] * p.scale_log2;
+              v[nt * 2 + e] = sv;
+              if (need_mask) {
+                const int kcol = key0 + nt * 8 + (lane & 3) * 2 + e;
+                const int pos = kpos_base + kcol;
+                const bool ok = is_new ? (kcol < p.n_qt && pos <= row_pos[mt][hf] && pos >= row_lo[mt][hf])
+                                       : (pos < b && pos >= row_lo[mt][hf]);
+                if (!ok) v[nt * 2 + e] = -INFINITY;
+              }
             }
           float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float m_new = fmaxf(m_r[mt][hf], mx);
-          const float moff = m_new == -INFINITY ? 0.f : m_new;
-          const float alpha = ex2_approx(m_r[mt][hf] - moff);  // 0 when the old max is -inf
-          m_r[mt][hf] = m_new;
+          // lazy rescale: move the offset only when the maximum grew by more than 2^8
+          if (mx > m_r[mt][hf] + 8.f) {
+            const float alpha = ex2_approx(m_r[mt][hf] - mx);  // 0 when the old offset is -inf
+            m_r[mt][hf] = mx;
+            l_r[mt][hf] *= alpha;
+#pragma unroll
+            for (int nd = 0; nd < D / 8; ++nd) {
+              o_acc[mt][nd][hf * 2 + 0] *= alpha;
+              o_acc[mt][nd][hf * 2 + 1] *= alpha;
+            }
+          }
+          const float moff = m_r[mt][hf] == -INFINITY ? 0.f : m_r[mt][hf];
           float pv[4];
-          float rs = 0.f;
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            pv[x] = ex2_approx(v[x] - moff);
-            rs += pv[x];
-          }
-          l_r[mt][hf] = l_r[mt][hf] * alpha + rs;
-#pragma unroll
-          for (int nd = 0; nd < D / 8; ++nd) {
-            o_acc[mt][nd][hf * 2 + 0] *= alpha;
-            o_acc[mt][nd][hf * 2 + 1] *= alpha;
-          }
+          for (int x = 0; x < 4; ++x) pv[x] = ex2_approx(v[x] - moff);
+          l_r[mt][hf] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
           // A fragment of P (16 rows x 16 keys): a0/a1 = keys 0-7 (rows r, r+8), a2/a3 = keys 8-15
           pa[mt][hf + 0] = pack_bf16x2(pv[0], pv[1]);
           pa[mt][hf + 2] = pack_bf16x2(pv[2], pv[3]);
@@ -412,7 +441,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           mma_bf16(o_acc[mt][nd2 * 2 + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b2, b3);
         }
       }
-      __syncthreads();  // the stage may be overwritten by the next iteration's loads
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 

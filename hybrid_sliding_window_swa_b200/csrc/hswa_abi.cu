@@ -363,6 +363,10 @@ int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa
     set_error("hybrid_decode_fwd: bad sizes (n_q_per_seq must be 1..8)");
     return HSWA_ERR_INVALID_ARG;
   }
+  if (max_ctx_len > 0x7fffffffLL - 4096) {
+    set_error("hybrid_decode_fwd: positions must stay below 2^31");
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
   if (n_seqs == 0) return HSWA_OK;
   const bool is_swa = layer < D.n_swa_layers;
   if (!q || !k_new || !v_new || !o || !ctx_len || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||

@@ -55,7 +55,7 @@ constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <=
 //                           0: read S twice (row maximum, then exponentials), fewer registers
 //  HSWA_SOFTMAX_REGS / HSWA_PRODUCER_REGS  setmaxnreg split (2 * 128 * a + 128 * b <= 384 * 168)
 #ifndef HSWA_POLY_PER8
-#define HSWA_POLY_PER8 2
+#define HSWA_POLY_PER8 0
 #endif
 #ifndef HSWA_SOFTMAX_SINGLE_PASS
 #define HSWA_SOFTMAX_SINGLE_PASS 1
