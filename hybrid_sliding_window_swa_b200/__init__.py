@@ -28,8 +28,11 @@ HSWA_ERR_DEVICE_BOUNDS = -6
 EXPORTED = [
     "kv_pool_layout", "kv_pool_create", "kv_pool_destroy", "kv_pool_append",
     "swa_prefill_fwd", "full_prefill_fwd", "hybrid_decode_workspace_size", "hybrid_decode_fwd",
-    "window_safe_len", "hswa_pool_check_error", "hswa_last_error",
+    "window_safe_len", "hswa_pool_check_error", "hswa_last_error", "hybrid_decode_fwd_noalloc",
 ]
+
+# scratch bytes available to hybrid_decode_fwd_noalloc (HSWA_NOALLOC_SCRATCH_BYTES in hswa.h)
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class HswaError(RuntimeError):
@@ -71,6 +74,7 @@ def load_library(path: str | None = None):
         "hybrid_decode_fwd": [p, i32, p, p, p, p, i32, i32, p, i64, p, p, i32, i32, p, sz, p],
         "window_safe_len": [p, p, p, ctypes.c_int32, ctypes.c_int32, p, p],
         "hswa_pool_check_error": [p, ctypes.POINTER(ctypes.c_int)],
+        "hybrid_decode_fwd_noalloc": [p, i32, p, p, p, p, i32, i32, p, i64, p, p, i32, i32, p],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -282,3 +286,20 @@ def hswa_pool_check_error(pool: KVPool) -> int:
 
 def hswa_last_error() -> str:
     return load_library().hswa_last_error().decode(errors="replace")
+
+
+def hybrid_decode_fwd_noalloc(pool: KVPool, layer: int, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                              ctx_len: torch.Tensor, max_ctx_len: int, o: torch.Tensor,
+                              seq_ids: torch.Tensor | None = None, page_table: torch.Tensor | None = None,
+                              stream=None) -> torch.Tensor:
+    """hybrid_decode_fwd for callers that cannot allocate device memory at call time: the split-KV
+    scratch is the library's fixed built-in array, so the caller passes only inputs and the output.
+    Calls that overlap on the GPU share that array and race; run them one after another."""
+    n_seqs, n_qt, hq, _ = q.shape
+    pt_stride = page_table.shape[1] if page_table is not None else 0
+    _check(load_library().hybrid_decode_fwd_noalloc(
+        pool.handle, layer, _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(o, torch.bfloat16, "o"), n_seqs, n_qt,
+        _ptr(ctx_len, torch.int64, "ctx_len"), max_ctx_len, _ptr(seq_ids, torch.int32, "seq_ids"),
+        _ptr(page_table, torch.int32, "page_table"), pt_stride, hq, _stream(stream)))
+    return o

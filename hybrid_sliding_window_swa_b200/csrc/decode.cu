@@ -18,6 +18,8 @@
 // memory at the end of the item. Items with one split write the output directly; the
 // others write (m, l, O) partials that merge_kernel combines:
 //   o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -658,3 +660,111 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
 }
 
 }  // namespace hswa
+
+// ---------------------------------------------------------------- decode without a workspace
+
+// The scratch of hybrid_decode_fwd_noalloc: one fixed array in device memory, reserved on
+// every GPU that loads this library and held until the process exits. Host code cannot use
+// this name as a device address; the address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HSWA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on first use).
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    hswa::set_error("hybrid_decode_fwd_noalloc: no usable current device (%s)",
+                    e == cudaSuccess ? "device index out of range" : cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr) {
+      hswa::set_error("hybrid_decode_fwd_noalloc: looking up the scratch array failed: %s",
+                      cudaGetErrorString(e));
+      return HSWA_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return HSWA_OK;
+}
+}  // namespace
+
+extern "C" int hybrid_decode_fwd_noalloc(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
+                                         const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq,
+                                         const int64_t* ctx_len, int64_t max_ctx_len, const int32_t* seq_ids,
+                                         const int32_t* page_table, int pt_stride, int n_q_heads, void* stream) {
+  using hswa::set_error;
+  if (!pool) {
+    set_error("hybrid_decode_fwd_noalloc: null pool");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  if (layer < 0 || layer >= D.n_swa_layers + D.n_full_layers) {
+    set_error("hybrid_decode_fwd_noalloc: layer %d out of range", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const int hkv = D.n_kv_heads;
+  if (n_q_heads < 1 || n_q_heads % hkv != 0 || n_q_heads / hkv > 16) {
+    set_error("hybrid_decode_fwd_noalloc: n_q_heads %d must be a positive multiple of n_kv_heads %d (ratio <= 16)",
+              n_q_heads, hkv);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (n_seqs < 0 || n_q_per_seq < 1 || n_q_per_seq > 8 || max_ctx_len < 0) {
+    set_error("hybrid_decode_fwd_noalloc: bad sizes (n_q_per_seq must be 1..8)");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (max_ctx_len > 0x7fffffffLL - 4096) {
+    set_error("hybrid_decode_fwd_noalloc: positions must stay below 2^31");
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (n_seqs == 0) return HSWA_OK;
+  const bool is_swa = layer < D.n_swa_layers;
+  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
+  if (!q || !k_new || !v_new || !o || !ctx_len || misaligned(q) || misaligned(k_new) || misaligned(v_new) ||
+      misaligned(o) || (is_swa && !seq_ids) || (!is_swa && (!page_table || pt_stride < 1))) {
+    set_error("hybrid_decode_fwd_noalloc: missing or misaligned device pointer");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const size_t need = hswa::decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, hkv, D.head_dim,
+                                                   is_swa ? D.window : 0, max_ctx_len);
+  if (need > (size_t)HSWA_NOALLOC_SCRATCH_BYTES) {
+    set_error("hybrid_decode_fwd_noalloc: this call needs %zu bytes of scratch but the built-in array holds %zu; "
+              "use hybrid_decode_fwd with a caller-provided workspace",
+              need, (size_t)HSWA_NOALLOC_SCRATCH_BYTES);
+    return HSWA_ERR_OUT_OF_MEMORY;
+  }
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  hswa::DecodeLaunch L{};
+  L.n_seqs = n_seqs;
+  L.n_qt = n_q_per_seq;
+  L.Hq = n_q_heads;
+  L.Hkv = hkv;
+  L.d = D.head_dim;
+  L.window = is_swa ? D.window : 0;
+  L.q = q;
+  L.k_new = k_new;
+  L.v_new = v_new;
+  L.o = o;
+  L.ctx_len = ctx_len;
+  L.max_ctx_len = max_ctx_len;
+  L.seq_ids = seq_ids;
+  L.page_table = page_table;
+  L.pt_stride = pt_stride;
+  L.pool = pool;
+  L.ring_layer = is_swa ? layer : 0;
+  L.full_layer = is_swa ? 0 : layer - D.n_swa_layers;
+  L.workspace = scratch;
+  L.ws_bytes = (size_t)HSWA_NOALLOC_SCRATCH_BYTES;
+  return hswa::launch_decode(L, static_cast<cudaStream_t>(stream));
+}

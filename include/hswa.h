@@ -28,8 +28,9 @@
  *    device (a page id out of range, a context length above the declared
  *    maximum, a wait that ran out) are recorded in the pool's device error word
  *    and read back with hswa_pool_check_error().
- *  - The library never allocates device memory. Pool memory and the decode
- *    workspace are passed in by the caller.
+ *  - The library never allocates device memory per call. Pool memory and the decode
+ *    workspace are passed in by the caller (hybrid_decode_fwd_noalloc instead uses one
+ *    fixed scratch array that is reserved when the library's device code is loaded).
  *  - Supported shapes: head_dim 64 or 128, n_q_heads a multiple of n_kv_heads,
  *    n_q_heads / n_kv_heads <= 16, W >= 1, page_size 64. Anything else returns
  *    HSWA_ERR_UNSUPPORTED_SHAPE.
@@ -167,6 +168,29 @@ HSWA_API int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, c
                       const int64_t* ctx_len, int64_t max_ctx_len, const int32_t* seq_ids,
                       const int32_t* page_table, int pt_stride, int n_q_heads, void* workspace,
                       size_t ws_bytes, void* stream);
+
+/* Largest scratch hybrid_decode_fwd_noalloc can use: 64 MiB. */
+#define HSWA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* hybrid_decode_fwd without a workspace argument. The source pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory when they call
+ * the library -- for example a plugin inside a host runtime that owns every device
+ * allocation, or a serving loop that must not call cudaMalloc (an allocation can
+ * synchronise the device). Its scratch is one fixed device array of
+ * HSWA_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that loads the library
+ * keeps until the process exits; nothing is allocated per call.
+ *  - Same arguments, layouts and results as hybrid_decode_fwd, minus workspace/ws_bytes.
+ *  - Returns HSWA_ERR_OUT_OF_MEMORY, before launching anything, when the call would need
+ *    more scratch than the array holds (hybrid_decode_workspace_size() reports the need).
+ *  - The first call on a device looks up the array's device address on the current
+ *    device; make that first call before any stream capture.
+ *  - All calls on a device share the one array: calls that overlap on the GPU (other
+ *    streams, other host threads) race and give wrong results; serialise them. Leftover
+ *    contents from an earlier call do not matter (the kernels reset what they read). */
+HSWA_API int hybrid_decode_fwd_noalloc(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
+                                       const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq,
+                                       const int64_t* ctx_len, int64_t max_ctx_len, const int32_t* seq_ids,
+                                       const int32_t* page_table, int pt_stride, int n_q_heads, void* stream);
 
 /* Window-safe prefix-match length ("MiMo v2.5 inference optimisation", section
  * "KV cache redesign": a prefix-cache match may be reused only as far as the
