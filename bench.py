@@ -119,11 +119,18 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Largest value over all ranks (the step time of a weak-scaling run is the slowest rank's)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, ws: int, ms_max: float, scale: float) -> float:
+    """Whole-job throughput: every rank processes the same units; time is the slowest rank's."""
+    return units_per_rank * ws / ms_max / scale
 
 
 def barrier(ws):
@@ -336,6 +343,141 @@ class LongContext1M:
         return dt, 4 * self.d * done * self.W * self.Hq, done
 
 
+class DecodeBatch:
+    """Hybrid decode step: n sequences with context lengths log-uniform in [1K, 256K], 4 query
+    tokens each (1 + 3 multi-token-prediction drafts), 6 SWA layers on a 128-slot ring and 1 full
+    layer on 64-token pages (seeded random page permutation), Hq=64, Hkv=8, d=128, bf16 N(0,1).
+    One step = the 7 hybrid_decode_fwd calls. The metric counts the bytes the step must read
+    (K/V of every cached key in every window, plus Q, the new K/V and O)."""
+    launches_per_step = 7 * 3  # plan + decode (+ merge on the full layer) per call
+
+    def __init__(self, hs, n=256, seq_offset=0, Hq=64, Hkv=8, d=128, W=128, nq=4, n_swa=6):
+        self.hs = hs
+        dev = "cuda"
+        self.n, self.Hq, self.Hkv, self.d, self.W, self.nq, self.n_swa = n, Hq, Hkv, d, W, nq, n_swa
+        self.name = f"hybrid_decode_{n}seq_L1K-256K_6swa_1full_Hq64_Hkv8_d128_4tok"
+        self.base = 200 + seq_offset * 100000
+        u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 4, seq_offset), n)
+        self.lens = torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
+        lens = self.lens
+        self.S = int(lens.sum())
+        pps = (lens + nq + 63) // 64
+        total_pages = int(pps.sum())
+        maxp = int(pps.max())
+        self.pool = hs.kv_pool_create(hs.PoolDesc(n_swa, 1, W, Hkv, d, n, total_pages))
+        perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 5, seq_offset), total_pages).to(torch.int32)
+        pt = torch.zeros(n, maxp, dtype=torch.int32)
+        off = 0
+        for i in range(n):
+            pt[i, :pps[i]] = perm[off:off + int(pps[i])]
+            off += int(pps[i])
+        self.pt = pt.to(dev)
+        self.sid = torch.arange(n, dtype=torch.int32, device=dev)
+        self.full_layer = n_swa
+        for b in range(n):
+            L = int(lens[b])
+            for c0 in range(0, L, 65536):
+                m = min(65536, L - c0)
+                k = gen(synth.TAG_K, self.full_layer, self.base + b, c0, m, Hkv, d, 1.0, dev)[None]
+                v = gen(synth.TAG_V, self.full_layer, self.base + b, c0, m, Hkv, d, 1.0, dev)[None]
+                hs.kv_pool_append(self.pool, self.full_layer, k, v, torch.tensor([c0], device=dev),
+                                  page_table=self.pt[b:b + 1])
+            for layer in range(n_swa):
+                k = gen(synth.TAG_K, layer, self.base + b, L - W, W, Hkv, d, 1.0, dev)[None]
+                v = gen(synth.TAG_V, layer, self.base + b, L - W, W, Hkv, d, 1.0, dev)[None]
+                hs.kv_pool_append(self.pool, layer, k, v, torch.tensor([L - W], device=dev), seq_ids=self.sid[b:b + 1])
+        self.ctx = lens.to(dev)
+        self.maxL = int(lens.max())
+        self.qs, self.kn, self.vn = [], [], []
+        for layer in range(n_swa + 1):
+            self.qs.append(torch.stack([gen(synth.TAG_Q, layer, self.base + b, int(lens[b]), nq, Hq, d, 1.0, dev)
+                                        for b in range(n)]))
+            self.kn.append(torch.stack([gen(synth.TAG_K, layer, self.base + b, int(lens[b]), nq, Hkv, d, 1.0, dev)
+                                        for b in range(n)]))
+            self.vn.append(torch.stack([gen(synth.TAG_V, layer, self.base + b, int(lens[b]), nq, Hkv, d, 1.0, dev)
+                                        for b in range(n)]))
+        self.ws = torch.empty(hs.hybrid_decode_workspace_size(self.pool, n, nq, Hq, self.maxL), dtype=torch.uint8,
+                              device=dev)
+        self.outs = [torch.empty_like(self.qs[0]) for _ in range(n_swa + 1)]
+        self.kv_full = self.S * Hkv * d * 2 * 2
+        self.kv_swa = n_swa * n * (W - 1) * Hkv * d * 2 * 2
+        qo = n * nq * (Hq * 2 + Hkv * 2) * d * 2      # Q + O + new K + new V per layer
+        self.bytes = self.kv_full + self.kv_swa + (n_swa + 1) * qo
+        self.full_bytes_per_launch = self.kv_full + qo
+        torch.cuda.synchronize()
+
+    def step(self, ev=None):
+        hs = self.hs
+        for layer in range(self.n_swa):
+            hs.hybrid_decode_fwd(self.pool, layer, self.qs[layer], self.kn[layer], self.vn[layer], self.ctx, self.maxL,
+                                 self.ws, seq_ids=self.sid, o=self.outs[layer])
+        if ev is not None:
+            ev.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+            ev[-1][0].record()
+        L = self.full_layer
+        hs.hybrid_decode_fwd(self.pool, L, self.qs[L], self.kn[L], self.vn[L], self.ctx, self.maxL, self.ws,
+                             page_table=self.pt, o=self.outs[L])
+        if ev is not None:
+            ev[-1][1].record()
+
+    def e2e_setup(self):
+        self.h_in = [(q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory())
+                     for q, k, v in zip(self.qs, self.kn, self.vn)]
+        self.h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
+        self.h2d = sum((q.numel() + k.numel() + v.numel()) * 2 for q, k, v in self.h_in)
+        self.d2h = sum(o.numel() * 2 for o in self.h_out)
+
+    def e2e_step(self):
+        for (hq, hk, hv), q, k, v in zip(self.h_in, self.qs, self.kn, self.vn):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+        self.step()
+        for ho, o in zip(self.h_out, self.outs):
+            ho.copy_(o, non_blocking=True)
+
+    def check_sample(self, oracle):
+        """All rows of the two shortest sequences on the full layer and of two sequences on an SWA layer."""
+        lens, nq, Hq, Hkv, d, W = self.lens, self.nq, self.Hq, self.Hkv, self.d, self.W
+        order = torch.argsort(lens)
+        errs = []
+        for b in [int(order[0]), int(order[1])]:
+            L = int(lens[b])
+            k = gen(synth.TAG_K, self.full_layer, self.base + b, 0, L + nq, Hkv, d, 1.0, "cpu")
+            v = gen(synth.TAG_V, self.full_layer, self.base + b, 0, L + nq, Hkv, d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, self.full_layer, self.base + b, L, nq, Hq, d, 1.0, "cpu")
+            ref = oracle.attention(q, L + np.arange(nq), k, v, 0)
+            errs.append(np.abs(self.outs[self.full_layer][b].float().cpu().double().numpy() - ref).ravel())
+        for b in [int(order[-1]), min(7, self.n - 1)]:
+            L = int(lens[b])
+            k = gen(synth.TAG_K, 2, self.base + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
+            v = gen(synth.TAG_V, 2, self.base + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, 2, self.base + b, L, nq, Hq, d, 1.0, "cpu")
+            ref = oracle.attention(q, L + np.arange(nq), k, v, W, key_base=L - W + 1)
+            errs.append(np.abs(self.outs[2][b].float().cpu().double().numpy() - ref).ravel())
+        e = np.concatenate(errs)
+        return float(e.max()), float(e.mean())
+
+    def oracle_sample(self, oracle, budget_s=10.0, threads=None):
+        """Time the oracle on whole sequences of the full layer, shortest first, until about budget_s;
+        returns (seconds, bytes of K/V those rows read, sequences)."""
+        order = torch.argsort(self.lens)
+        dt, byts, done = 0.0, 0, 0
+        for b in order.tolist():
+            if dt >= budget_s:
+                break
+            L = int(self.lens[b])
+            k = gen(synth.TAG_K, self.full_layer, self.base + b, 0, L + self.nq, self.Hkv, self.d, 1.0, "cpu")
+            v = gen(synth.TAG_V, self.full_layer, self.base + b, 0, L + self.nq, self.Hkv, self.d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, self.full_layer, self.base + b, L, self.nq, self.Hq, self.d, 1.0, "cpu")
+            t0 = time.perf_counter()
+            oracle.attention(q, L + np.arange(self.nq), k, v, 0, n_threads=threads)
+            dt += time.perf_counter() - t0
+            byts += (L + self.nq) * self.Hkv * self.d * 2 * 2
+            done += 1
+        return dt, byts, done
+
+
 def secondary_results(hs, oracle_mod, hbm, bf16):
     out = []
     dev = "cuda"
@@ -426,102 +568,33 @@ def secondary_results(hs, oracle_mod, hbm, bf16):
 
 def decode_results(hs, oracle_mod, hbm):
     dev = "cuda"
-    n, Hq, Hkv, d, W, nq = 256, 64, 8, 128, 128, 4
-    u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 4), n)
-    lens = torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
-    S = int(lens.sum())
-    pps = (lens + nq + 63) // 64
-    total_pages = int(pps.sum())
-    maxp = int(pps.max())
-    n_swa = 6
-    pool = hs.kv_pool_create(hs.PoolDesc(n_swa, 1, W, Hkv, d, n, total_pages))
-    perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 5), total_pages).to(torch.int32)
-    pt = torch.zeros(n, maxp, dtype=torch.int32)
-    off = 0
-    for i in range(n):
-        pt[i, :pps[i]] = perm[off:off + int(pps[i])]
-        off += int(pps[i])
-    pt = pt.to(dev)
-    sid = torch.arange(n, dtype=torch.int32, device=dev)
-    full_layer = n_swa
-    for b in range(n):
-        L = int(lens[b])
-        for c0 in range(0, L, 65536):
-            m = min(65536, L - c0)
-            k = gen(synth.TAG_K, full_layer, 200 + b, c0, m, Hkv, d, 1.0, dev)[None]
-            v = gen(synth.TAG_V, full_layer, 200 + b, c0, m, Hkv, d, 1.0, dev)[None]
-            hs.kv_pool_append(pool, full_layer, k, v, torch.tensor([c0], device=dev), page_table=pt[b:b + 1])
-        for layer in range(n_swa):
-            k = gen(synth.TAG_K, layer, 200 + b, L - W, W, Hkv, d, 1.0, dev)[None]
-            v = gen(synth.TAG_V, layer, 200 + b, L - W, W, Hkv, d, 1.0, dev)[None]
-            hs.kv_pool_append(pool, layer, k, v, torch.tensor([L - W], device=dev), seq_ids=sid[b:b + 1])
-    ctx = lens.to(dev)
-    maxL = int(lens.max())
-    qs, kn, vn = [], [], []
-    for layer in range(n_swa + 1):
-        qs.append(torch.stack([gen(synth.TAG_Q, layer, 200 + b, int(lens[b]), nq, Hq, d, 1.0, dev) for b in range(n)]))
-        kn.append(torch.stack([gen(synth.TAG_K, layer, 200 + b, int(lens[b]), nq, Hkv, d, 1.0, dev) for b in range(n)]))
-        vn.append(torch.stack([gen(synth.TAG_V, layer, 200 + b, int(lens[b]), nq, Hkv, d, 1.0, dev) for b in range(n)]))
-    ws = torch.empty(hs.hybrid_decode_workspace_size(pool, n, nq, Hq, maxL), dtype=torch.uint8, device=dev)
-    outs = [torch.empty_like(qs[0]) for _ in range(n_swa + 1)]
-
-    def step():
-        for layer in range(n_swa):
-            hs.hybrid_decode_fwd(pool, layer, qs[layer], kn[layer], vn[layer], ctx, maxL, ws, seq_ids=sid,
-                                 o=outs[layer])
-        hs.hybrid_decode_fwd(pool, full_layer, qs[n_swa], kn[n_swa], vn[n_swa], ctx, maxL, ws, page_table=pt,
-                             o=outs[n_swa])
-
+    W = 128
+    wl = DecodeBatch(hs)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(2):
-        step()
+        wl.step()
     torch.cuda.synchronize()
     times, times_full = [], []
     for _ in range(5):
         flush.zero_()
-        a, b_, c = (torch.cuda.Event(True) for _ in range(3))
+        ev = []
+        a = torch.cuda.Event(True)
         a.record()
-        for layer in range(n_swa):
-            hs.hybrid_decode_fwd(pool, layer, qs[layer], kn[layer], vn[layer], ctx, maxL, ws, seq_ids=sid,
-                                 o=outs[layer])
-        b_.record()
-        hs.hybrid_decode_fwd(pool, full_layer, qs[n_swa], kn[n_swa], vn[n_swa], ctx, maxL, ws, page_table=pt,
-                             o=outs[n_swa])
-        c.record()
+        wl.step(ev)
         torch.cuda.synchronize()
-        times.append(a.elapsed_time(c))
-        times_full.append(b_.elapsed_time(c))
+        times.append(a.elapsed_time(ev[-1][1]))
+        times_full.append(ev[-1][0].elapsed_time(ev[-1][1]))
     ms = statistics.median(times)
     ms_full = statistics.median(times_full)
-    kv_full = S * Hkv * d * 2 * 2
-    kv_swa = n_swa * n * (W - 1) * Hkv * d * 2 * 2
-    qo = (n_swa + 1) * n * nq * (Hq * 2 + Hkv * 2) * d * 2
-    total_bytes = kv_full + kv_swa + qo
-    assert hs.hswa_pool_check_error(pool) == 0
-    # sampled parity: the two shortest sequences (full layer) and two sequences of one SWA layer
-    order = torch.argsort(lens)
-    errs = []
-    for b in [int(order[0]), int(order[1])]:
-        L = int(lens[b])
-        k = gen(synth.TAG_K, full_layer, 200 + b, 0, L + nq, Hkv, d, 1.0, "cpu")
-        v = gen(synth.TAG_V, full_layer, 200 + b, 0, L + nq, Hkv, d, 1.0, "cpu")
-        q = gen(synth.TAG_Q, full_layer, 200 + b, L, nq, Hq, d, 1.0, "cpu")
-        ref = oracle_mod.attention(q, L + np.arange(nq), k, v, 0)
-        errs.append(np.abs(outs[n_swa][b].float().cpu().double().numpy() - ref).ravel())
-    for b in [int(order[-1]), 7]:
-        L = int(lens[b])
-        k = gen(synth.TAG_K, 2, 200 + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
-        v = gen(synth.TAG_V, 2, 200 + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
-        q = gen(synth.TAG_Q, 2, 200 + b, L, nq, Hq, d, 1.0, "cpu")
-        ref = oracle_mod.attention(q, L + np.arange(nq), k, v, W, key_base=L - W + 1)
-        errs.append(np.abs(outs[2][b].float().cpu().double().numpy() - ref).ravel())
-    e = np.concatenate(errs)
-    res = [{"workload": "hybrid_decode_256seq_L1K-256K_6swa_1full_Hq64_Hkv8_d128_4tok", "metric": "hybrid decode KV GB/s",
-            "unit": "GB/s", "value": round(total_bytes / ms / 1e6, 1), "ms": round(ms, 3),
-            "pct_hbm_peak": round(100 * total_bytes / ms / 1e6 / hbm, 1), "bytes": total_bytes, "sum_ctx": S,
-            "full_layer_ms": round(ms_full, 3), "full_layer_gbs": round((kv_full + qo / 7) / ms_full / 1e6, 1),
-            "l2": "flushed (256 MiB write) before each step", "max_abs_err": float(e.max()),
-            "mean_abs_err": float(e.mean())}]
+    assert hs.hswa_pool_check_error(wl.pool) == 0
+    mx, mean = wl.check_sample(oracle_mod)
+    res = [{"workload": wl.name, "metric": "hybrid decode KV GB/s",
+            "unit": "GB/s", "value": round(wl.bytes / ms / 1e6, 1), "ms": round(ms, 3),
+            "pct_hbm_peak": round(100 * wl.bytes / ms / 1e6 / hbm, 1), "bytes": wl.bytes, "sum_ctx": wl.S,
+            "full_layer_ms": round(ms_full, 3), "full_layer_gbs": round(wl.full_bytes_per_launch / ms_full / 1e6, 1),
+            "l2": "flushed (256 MiB write) before each step", "max_abs_err": mx, "mean_abs_err": mean}]
+    del wl
+    torch.cuda.empty_cache()
     # window_safe_len over 4096 requests (bit-exact vs oracle)
     nr = 4096
     C = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 11), nr, 0, 262144)
@@ -550,8 +623,6 @@ def decode_results(hs, oracle_mod, hbm):
     ref = oracle_mod.window_safe_len(M.numpy(), C.numpy(), bits, W)
     res.append({"workload": "window_safe_len_4096req_W128", "metric": "latency", "unit": "us", "value": round(us, 2),
                 "requests_per_s": round(nr / (us * 1e-6)), "bit_exact": bool(np.array_equal(outw.cpu().numpy(), ref))})
-    del pool
-    torch.cuda.empty_cache()
     return res
 
 
@@ -622,7 +693,9 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", default="hswa", choices=["hswa", "reference"])
-    ap.add_argument("--workload", default="swa_prefill_16k", choices=["swa_prefill_16k", "long_context_1m"])
+    ap.add_argument("--workload", default="swa_prefill_16k",
+                    choices=["swa_prefill_16k", "long_context_1m", "hybrid_decode"])
+    ap.add_argument("--decode-seqs", type=int, default=256, help="sequences in the hybrid_decode batch")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -644,11 +717,18 @@ def main():
     import hybrid_sliding_window_swa_b200 as hs
     hs.load_library()
     hbm, bf16, bf16_sus, peak_src = peaks()
+    decode = args.workload == "hybrid_decode"
     if big:
         wl = LongContext1M(hs, seq_offset=rank)
         dominant_flops = wl.full_flops_per_launch
         peak = bf16_sus  # a seconds-long step: the sustained figure
         peak_name = f"{peak_src} bf16 sustained"
+    elif decode:
+        wl = DecodeBatch(hs, n=args.decode_seqs, seq_offset=rank)
+        wl.flops = wl.bytes  # the decode metric counts bytes
+        dominant_flops = wl.full_bytes_per_launch
+        peak = hbm
+        peak_name = f"{peak_src} HBM copy bandwidth"
     else:
         wl = SwaPrefill16k(hs, seq_offset=rank * 2)
         dominant_flops = wl.flops
@@ -680,8 +760,9 @@ def main():
     ms_step = e0.elapsed_time(e1) / args.steps
     kern_ms = sum(a.elapsed_time(b) for a, b in kern_events) / len(kern_events)
     ms_max = max_over_ranks(ms_step, ws)
-    value = wl.flops * ws / ms_max / 1e9  # TFLOP/s over all ranks
-    achieved = dominant_flops / kern_ms / 1e9
+    scale = 1e6 if decode else 1e9  # GB/s for the decode workload, TFLOP/s otherwise
+    value = weak_scaling_value(wl.flops, ws, ms_max, scale)
+    achieved = dominant_flops / kern_ms / scale
     assert hs.hswa_pool_check_error(wl.pool) == 0
 
     max_err, mean_err = (None, None)
@@ -702,10 +783,12 @@ def main():
         b.record()
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, ws)
-        e2e = {"value": round(wl.flops * ws / e2e_ms / 1e9, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
-               "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
-               "path": "pinned host Q/K/V -> device, swa_prefill_fwd + kv_pool_append via the Python binding "
-                       "(C ABI), O -> pinned host"}
+        e2e = {"value": round(wl.flops * ws / e2e_ms / scale, 2), "unit": "GB/s" if decode else "TFLOP/s",
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
+               "path": ("pinned host Q and new K/V of 7 layers -> device, 7 hybrid_decode_fwd calls via the Python "
+                        "binding (C ABI), O of 7 layers -> pinned host") if decode else
+                       ("pinned host Q/K/V -> device, swa_prefill_fwd + kv_pool_append via the Python binding "
+                        "(C ABI), O -> pinned host")}
     if rank == 0:
         import oracle
         oracle.build()
@@ -713,11 +796,16 @@ def main():
         if not args.no_cpu:
             threads = os.cpu_count() or 1
             dt, fl, nrows = wl.oracle_sample(oracle, threads=threads)
-            what = ("32 heads at the end of sequence 0 (full 4096-key windows)" if not big else
-                    "64 heads of SWA layer 3 (full 128-key windows)")
-            cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                   "sample": f"{nrows} query rows x {what}, fp64, {dt:.1f} s"}
-        if not args.no_secondary and ws == 1 and not big:
+            if decode:
+                cpu = {"value": fl / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                       "sample": f"all 4 x 64 rows of the {nrows} shortest sequences on the full layer, fp64, "
+                                 f"{dt:.1f} s"}
+            else:
+                what = ("32 heads at the end of sequence 0 (full 4096-key windows)" if not big else
+                        "64 heads of SWA layer 3 (full 128-key windows)")
+                cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                       "sample": f"{nrows} query rows x {what}, fp64, {dt:.1f} s"}
+        if not args.no_secondary and ws == 1 and not big and not decode:
             sec = secondary_results(hs, oracle, hbm, bf16)
 
     if rank == 0:
@@ -728,6 +816,13 @@ def main():
                       "l2": "inputs larger than L2 (each full layer reads 4 GiB of pages)",
                       "footprint": wl.footprint()}
             kname = "prefill_kernel<128> (full_prefill_fwd, one full layer)"
+        elif decode:
+            config = {"workload": wl.name, "n_seqs_per_gpu": wl.n, "sum_ctx": wl.S, "max_ctx": wl.maxL,
+                      "tokens_per_seq": wl.nq, "window": wl.W, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
+                      "layers": "6 SWA (ring) + 1 full (pages)", "parallelism": f"independent batches x{ws}",
+                      "step": "7 hybrid_decode_fwd calls", "bytes_per_step": wl.bytes,
+                      "l2": "inputs larger than L2 (tens of GB of K/V per step)"}
+            kname = "hybrid_decode_fwd on the full layer (plan_kernel + decode_kernel<128,2> + merge_kernel)"
         else:
             config = {"workload": wl.name, "B_per_gpu": wl.B, "seq_len": wl.N, "window": wl.W, "Hq": wl.Hq,
                       "Hkv": wl.Hkv, "head_dim": wl.d, "parallelism": f"independent batches x{ws}",
@@ -735,17 +830,18 @@ def main():
                       "l2": "inputs larger than L2 (Q 268 MB + K/V 134 MB + O 268 MB per step)"}
             kname = "prefill_kernel<128> (swa_prefill_fwd)"
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based normal, rounded to bf16)",
             "config": config,
-            "pct_bf16_peak": round(100 * value / ws / bf16, 1),
-            "roofline": {"bound": "tensor", "kernel": kname,
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            ("pct_hbm_peak" if decode else "pct_bf16_peak"): round(100 * value / ws / (hbm if decode else bf16), 1),
+            "roofline": {"bound": "hbm" if decode else "tensor", "kernel": kname,
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s" if decode else "TFLOP/s",
                          "frac": round(achieved / peak, 3), "peak_source": peak_name,
-                         "algorithmic_flops_per_launch": dominant_flops, "kernel_ms": round(kern_ms, 4),
-                         "traffic": stored_traffic(args.workload)},
+                         ("algorithmic_bytes_per_launch" if decode else "algorithmic_flops_per_launch"): dominant_flops,
+                         "kernel_ms": round(kern_ms, 4), "traffic": stored_traffic(args.workload)},
             "parity": {"max_abs_err": max_err, "mean_abs_err": mean_err},
             "gpu_launches": wl.launches_per_step * args.steps,
             "clocks": clk,
