@@ -516,7 +516,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
   }
 }
 
-// One CTA per (sequence, KV head) with more than one split.
+// One CTA of 256 threads per (sequence, KV head) with more than one split.
+//  phase 1: 8 threads per row reduce the splits' maxima M and denominators sum_c 2^(m_c - M) l_c
+//           (shuffles within the 8-thread group), keeping the factors 2^(m_c - M) in shared memory;
+//  phase 2: each thread owns 4 float4 groups of the R x D output and walks the splits with
+//           8 independent loads in flight.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
   const int g = blockIdx.x % p.Hkv;
@@ -528,39 +532,90 @@ __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
   extern __shared__ float msh[];  // [nsp][R] scale factors, then [R] inverse denominators
   float* fac = msh;
   float* inv = msh + (size_t)nsp * p.R;
-  for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+  const uint8_t* part0 = p.ws + p.part_off + (size_t)(c0 * p.Hkv + g) * p.part_bytes;
+  const size_t split_stride = (size_t)p.Hkv * p.part_bytes;  // consecutive splits of this (s, g)
+  const int lane8 = threadIdx.x & 7;
+  // rows padded to whole warps (4 rows of 8 threads per warp) so every shuffle has all 32 lanes
+  const int r_pad = (p.R + 3) & ~3;
+  for (int r = threadIdx.x >> 3; r < r_pad; r += 32) {
+    const bool live = r < p.R;
     float M = -INFINITY;
-    for (int c = 0; c < nsp; ++c) {
-      const float* part =
-          reinterpret_cast<const float*>(p.ws + p.part_off + (size_t)((c0 + c) * p.Hkv + g) * p.part_bytes);
-      M = fmaxf(M, part[p.R * D + r]);
-    }
+    for (int c = lane8; live && c < nsp; c += 8)
+      M = fmaxf(M, reinterpret_cast<const float*>(part0 + c * split_stride)[p.R * D + r]);
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 4));
     const float Mo = M == -INFINITY ? 0.f : M;
     float den = 0.f;
-    for (int c = 0; c < nsp; ++c) {
-      const float* part =
-          reinterpret_cast<const float*>(p.ws + p.part_off + (size_t)((c0 + c) * p.Hkv + g) * p.part_bytes);
+    for (int c = lane8; live && c < nsp; c += 8) {
+      const float* part = reinterpret_cast<const float*>(part0 + c * split_stride);
       const float f = ex2_approx(part[p.R * D + r] - Mo);
       fac[c * p.R + r] = f;
       den += f * part[p.R * D + p.R + r];
     }
-    inv[r] = 1.f / den;
+    den += __shfl_xor_sync(0xffffffffu, den, 1);
+    den += __shfl_xor_sync(0xffffffffu, den, 2);
+    den += __shfl_xor_sync(0xffffffffu, den, 4);
+    if (live && lane8 == 0) inv[r] = 1.f / den;
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < p.R * (D / 2); idx += blockDim.x) {
-    const int r = idx / (D / 2), col = (idx % (D / 2)) * 2;
-    float x0 = 0.f, x1 = 0.f;
-    for (int c = 0; c < nsp; ++c) {
-      const float* part =
-          reinterpret_cast<const float*>(p.ws + p.part_off + (size_t)((c0 + c) * p.Hkv + g) * p.part_bytes);
-      const float2 v = *reinterpret_cast<const float2*>(part + r * D + col);
-      const float f = fac[c * p.R + r];
-      x0 += f * v.x;
-      x1 += f * v.y;
+  constexpr int Q4 = D / 4;  // float4 groups per row
+  const int n_items = p.R * Q4;
+  for (int base = threadIdx.x; base < n_items; base += 4 * blockDim.x) {
+    float4 acc[4];
+    int it_r[4], it_c[4];
+    bool ok[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * blockDim.x;
+      ok[u] = idx < n_items;
+      it_r[u] = ok[u] ? idx / Q4 : 0;
+      it_c[u] = ok[u] ? (idx % Q4) * 4 : 0;
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const int t = r / p.G, hh = r % p.G;
-    uint16_t* dst = p.o + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + col;
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(x0 * inv[r], x1 * inv[r]);
+    int c = 0;
+    for (; c + 2 <= nsp; c += 2) {
+      const float* pa = reinterpret_cast<const float*>(part0 + c * split_stride);
+      const float* pb = reinterpret_cast<const float*>(part0 + (c + 1) * split_stride);
+      float4 va[4], vb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        va[u] = *reinterpret_cast<const float4*>(pa + it_r[u] * D + it_c[u]);
+        vb[u] = *reinterpret_cast<const float4*>(pb + it_r[u] * D + it_c[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float fa = fac[c * p.R + it_r[u]], fb = fac[(c + 1) * p.R + it_r[u]];
+        acc[u].x += fa * va[u].x + fb * vb[u].x;
+        acc[u].y += fa * va[u].y + fb * vb[u].y;
+        acc[u].z += fa * va[u].z + fb * vb[u].z;
+        acc[u].w += fa * va[u].w + fb * vb[u].w;
+      }
+    }
+    if (c < nsp) {
+      const float* pa = reinterpret_cast<const float*>(part0 + c * split_stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 va = *reinterpret_cast<const float4*>(pa + it_r[u] * D + it_c[u]);
+        const float fa = fac[c * p.R + it_r[u]];
+        acc[u].x += fa * va.x;
+        acc[u].y += fa * va.y;
+        acc[u].z += fa * va.z;
+        acc[u].w += fa * va.w;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!ok[u]) continue;
+      const int r = it_r[u];
+      const float iv = inv[r];
+      const int t = r / p.G, hh = r % p.G;
+      uint16_t* dst = p.o + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + it_c[u];
+      uint2 pk;
+      pk.x = pack_bf16x2(acc[u].x * iv, acc[u].y * iv);
+      pk.y = pack_bf16x2(acc[u].z * iv, acc[u].w * iv);
+      *reinterpret_cast<uint2*>(dst) = pk;
+    }
   }
 }
 
