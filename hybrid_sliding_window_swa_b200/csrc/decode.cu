@@ -30,7 +30,11 @@ namespace {
 constexpr int DEC_THREADS = 128;
 constexpr int KB = 64;          // keys per block
 constexpr int NST = 3;          // pipeline stages
-constexpr int SPLIT = 4096;     // cached keys per split (multiple of KB)
+#ifndef HSWA_DECODE_SPLIT
+#define HSWA_DECODE_SPLIT 8192
+#endif
+constexpr int SPLIT = HSWA_DECODE_SPLIT;  // cached keys per split (tuning parameter, multiple of KB)
+static_assert(SPLIT % 64 == 0, "splits start on page boundaries");
 
 struct WsHeader {
   int counter;
@@ -387,24 +391,27 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       const int kpos_base = is_new ? L : a + kb2 * KB;
       const bool need_mask = is_new || kpos_base + KB > b || kpos_base < lo_max;
       uint32_t pa[MT][4];
+      // this lane's key columns are key0 + (lane & 3) * 2 + {0, 1, 8, 9}
+      const int col_base = kpos_base + key0 + (lane & 3) * 2;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           float v[4];
+          // allowed offsets j (key = col_base + j) for this row: lo_j <= j < hi_j
+          int lo_j = 0, hi_j = 16;
+          if (need_mask) {
+            const int hi_pos = is_new ? min(L + p.n_qt, row_pos[mt][hf] + 1) : b;  // exclusive
+            lo_j = row_lo[mt][hf] - col_base;
+            hi_j = hi_pos - col_base;
+          }
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
+              const int j = nt * 8 + e;
               const float sv = sacc[mt][nt][hf * 2 + e] * p.scale_log2;
-              v[nt * 2 + e] = sv;
-              if (need_mask) {
-                const int kcol = key0 + nt * 8 + (lane & 3) * 2 + e;
-                const int pos = kpos_base + kcol;
-                const bool ok = is_new ? (kcol < p.n_qt && pos <= row_pos[mt][hf] && pos >= row_lo[mt][hf])
-                                       : (pos < b && pos >= row_lo[mt][hf]);
-                if (!ok) v[nt * 2 + e] = -INFINITY;
-              }
+              v[nt * 2 + e] = (j >= lo_j && j < hi_j) ? sv : -INFINITY;
             }
           float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -461,9 +468,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           l_w[warp * ROWS + r] = lsum;
         }
       }
-    float* acc = reinterpret_cast<float*>(smem + SM::ACC_OFF);
+    // each warp's partial O, rescaled to the rows' common maximum, goes to its own region of the
+    // (now idle) K/V stage buffers; the output pass sums the four regions (no shared atomics)
+    constexpr int RS = D + 8;  // padded row stride: a warp's float2 stores hit distinct banks
+    float* part_w = reinterpret_cast<float*>(smem + SM::ACC_OFF);  // [4][ROWS][RS]
+    static_assert(4 * ROWS * RS * 4 <= 2 * NST * SM::TILE, "merge regions must fit in the K/V stages");
     __syncthreads();
-    for (int idx = tid; idx < ROWS * D; idx += DEC_THREADS) acc[idx] = 0.f;
     for (int r = tid; r < ROWS; r += DEC_THREADS) {
       float M = -INFINITY;
       for (int w = 0; w < 4; ++w) M = fmaxf(M, m_w[w * ROWS + r]);
@@ -481,32 +491,45 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
         const int r = mt * 16 + (lane >> 2) + hf * 8;
         const float Mo = m_all[r] == -INFINITY ? 0.f : m_all[r];
         const float f = ex2_approx(m_r[mt][hf] - Mo);
+        float* dst = part_w + (warp * ROWS + r) * RS + (lane & 3) * 2;
 #pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd) {
-          const int col = nd * 8 + (lane & 3) * 2;
-          atomicAdd(&acc[r * D + col], o_acc[mt][nd][hf * 2 + 0] * f);
-          atomicAdd(&acc[r * D + col + 1], o_acc[mt][nd][hf * 2 + 1] * f);
-        }
+        for (int nd = 0; nd < D / 8; ++nd)
+          *reinterpret_cast<float2*>(dst + nd * 8) =
+              make_float2(o_acc[mt][nd][hf * 2 + 0] * f, o_acc[mt][nd][hf * 2 + 1] * f);
       }
+    __syncthreads();
+    // element (r, c) of the merged, unnormalised O
+    auto merged4 = [&](int r, int c) -> float4 {
+      float4 x = *reinterpret_cast<const float4*>(part_w + (0 * ROWS + r) * RS + c);
+#pragma unroll
+      for (int w = 1; w < 4; ++w) {
+        const float4 y = *reinterpret_cast<const float4*>(part_w + (w * ROWS + r) * RS + c);
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      return x;
+    };
     __syncthreads();
     if (nsp == 1) {
       // single split: normalise and write bf16 output rows
       for (int idx = tid; idx < p.R * (D / 8); idx += DEC_THREADS) {
         const int r = idx / (D / 8), ch = idx % (D / 8);
         const float inv = 1.f / l_all[r];
-        const float* src = acc + r * D + ch * 8;
+        const float4 lo4 = merged4(r, ch * 8), hi4 = merged4(r, ch * 8 + 4);
         uint4 pk;
-        pk.x = pack_bf16x2(src[0] * inv, src[1] * inv);
-        pk.y = pack_bf16x2(src[2] * inv, src[3] * inv);
-        pk.z = pack_bf16x2(src[4] * inv, src[5] * inv);
-        pk.w = pack_bf16x2(src[6] * inv, src[7] * inv);
+        pk.x = pack_bf16x2(lo4.x * inv, lo4.y * inv);
+        pk.y = pack_bf16x2(lo4.z * inv, lo4.w * inv);
+        pk.z = pack_bf16x2(hi4.x * inv, hi4.y * inv);
+        pk.w = pack_bf16x2(hi4.z * inv, hi4.w * inv);
         const int t = r / p.G, hh = r % p.G;
         uint16_t* dst = p.o + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
         *reinterpret_cast<uint4*>(dst) = pk;
       }
     } else {
       float* part = reinterpret_cast<float*>(p.ws + p.part_off + (size_t)item * p.part_bytes);
-      for (int idx = tid; idx < p.R * D; idx += DEC_THREADS) part[idx] = acc[idx];
+      for (int idx = tid; idx < p.R * (D / 4); idx += DEC_THREADS) {
+        const int r = idx / (D / 4), c = (idx % (D / 4)) * 4;
+        *reinterpret_cast<float4*>(part + r * D + c) = merged4(r, c);
+      }
       for (int r = tid; r < p.R; r += DEC_THREADS) {
         part[p.R * D + r] = m_all[r];
         part[p.R * D + p.R + r] = l_all[r];
