@@ -29,6 +29,7 @@ EXPORTED = [
     "kv_pool_layout", "kv_pool_create", "kv_pool_destroy", "kv_pool_append",
     "swa_prefill_fwd", "full_prefill_fwd", "hybrid_decode_workspace_size", "hybrid_decode_fwd",
     "window_safe_len", "hswa_pool_check_error", "hswa_last_error", "hybrid_decode_fwd_noalloc",
+    "hswa_selftest_wait_timeout",
 ]
 
 # scratch bytes available to hybrid_decode_fwd_noalloc (HSWA_NOALLOC_SCRATCH_BYTES in hswa.h)
@@ -75,6 +76,7 @@ def load_library(path: str | None = None):
         "window_safe_len": [p, p, p, ctypes.c_int32, ctypes.c_int32, p, p],
         "hswa_pool_check_error": [p, ctypes.POINTER(ctypes.c_int)],
         "hybrid_decode_fwd_noalloc": [p, i32, p, p, p, p, i32, i32, p, i64, p, p, i32, i32, p],
+        "hswa_selftest_wait_timeout": [p, i64, p],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -282,6 +284,11 @@ def hswa_pool_check_error(pool: KVPool) -> int:
     code = ctypes.c_int()
     _check(load_library().hswa_pool_check_error(pool.handle, ctypes.byref(code)))
     return code.value
+
+
+def hswa_selftest_wait_timeout(pool: KVPool, limit_ns: int = 50_000_000, stream=None):
+    """Run one bounded wait that is meant to run out (see include/hswa.h)."""
+    _check(load_library().hswa_selftest_wait_timeout(pool.handle, limit_ns, _stream(stream)))
 
 
 def hswa_last_error() -> str:

@@ -419,6 +419,14 @@ int window_safe_len(const int64_t* match_len, const int64_t* cached_len, const u
                                 static_cast<cudaStream_t>(stream));
 }
 
+int hswa_selftest_wait_timeout(hswa_pool* pool, int64_t limit_ns, void* stream) {
+  if (!pool || limit_ns < 1000000 || limit_ns > 2000000000) {
+    set_error("hswa_selftest_wait_timeout: a pool and a limit of 1 ms .. 2 s are required");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  return launch_selftest_wait(pool->err, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream));
+}
+
 int hswa_pool_check_error(hswa_pool* pool, int* device_code) {
   if (!pool || !device_code) {
     set_error("hswa_pool_check_error: null argument");

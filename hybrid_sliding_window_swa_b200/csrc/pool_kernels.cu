@@ -146,4 +146,25 @@ int launch_window_safe_len(const int64_t* m, const int64_t* c, const uint32_t* v
   return HSWA_OK;
 }
 
+// One thread waits on a fresh mbarrier that nothing ever arrives at, through the same bounded
+// wait every kernel of the library uses; the wait gives up after limit_ns and records
+// HSWA_ERR_TIMEOUT in the error word, and the kernel returns normally.
+__global__ void selftest_wait_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  (void)mbar_wait_limit(&bar, 0, err, limit_ns);
+}
+
+int launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(err, limit_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("hswa_selftest_wait_timeout: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
 }  // namespace hswa

@@ -204,6 +204,12 @@ HSWA_API int window_safe_len(const int64_t* match_len, const int64_t* cached_len
                     const uint32_t* slot_valid, int32_t W, int32_t n_req, int64_t* out_len,
                     void* stream);
 
+/* Diagnostic: run, on `stream`, one wait on a barrier that nothing arrives at, through the same
+ * bounded wait every kernel uses, with a limit of limit_ns (1 ms .. 2 s; the kernels themselves
+ * use 2 s). The wait gives up, records HSWA_ERR_TIMEOUT in the pool's error word and the kernel
+ * returns; hswa_pool_check_error() then reports it. Nothing faults and the context stays usable. */
+HSWA_API int hswa_selftest_wait_timeout(hswa_pool* pool, int64_t limit_ns, void* stream);
+
 /* Synchronise the device, return the pool's device error word in *device_code
  * (0 if none, else a negative HSWA_ERR_* code) and clear it. */
 HSWA_API int hswa_pool_check_error(hswa_pool* pool, int* device_code);

@@ -65,7 +65,7 @@ def test_swa_decode_ring(W):
 
 
 @pytest.mark.parametrize("lens,n_qt,hq,hkv,d", [
-    ([0, 5, 64, 65, 4095, 4096, 4097, 9000], 4, 16, 2, 128),   # split boundaries at 4096
+    ([0, 5, 64, 65, 8191, 8192, 8193, 17000], 4, 16, 2, 128),  # split boundaries (8192-key splits)
     ([20000, 1, 12345], 4, 32, 4, 128),                         # 8 rows per KV head
     ([300, 5000], 1, 8, 1, 64),                                 # single token, MHA-like group of 8
     ([1024, 777, 50000], 2, 4, 4, 64),                          # G = 1
