@@ -343,6 +343,115 @@ class LongContext1M:
         return dt, 4 * self.d * done * self.W * self.Hq, done
 
 
+class HybridChunk131k:
+    """One 16K-token chunk after a 131072-token cached prefix (B=1, Hq=64, Hkv=8, d=128, bf16 N(0,1)):
+    kind 'swa' is the sliding-window layer (W=128; the 127 prefix keys it needs come from the
+    rolling buffer) -- bandwidth-bound, its metric is bytes moved; kind 'full' is the full layer
+    over all 147456 keys through a randomly permuted 64-token page table (the chunk appended
+    first) -- tensor-bound, its metric is useful FLOPs."""
+    launches_per_step = 1
+
+    def __init__(self, hs, kind="swa", seq_offset=0, P=131072, Nc=16384, W=128, Hq=64, Hkv=8, d=128):
+        self.hs, self.kind = hs, kind
+        self.P, self.Nc, self.W, self.Hq, self.Hkv, self.d = P, Nc, W, Hq, Hkv, d
+        self.N, self.B = Nc, 1
+        self.seq = 100 + seq_offset
+        self.name = ("swa_chunk16k_after_131072_W128_Hq64_Hkv8_d128" if kind == "swa" else
+                     "full_chunk16k_after_131072_paged_Hq64_Hkv8_d128")
+        dev = "cuda"
+        total = P + Nc
+        pages = total // 64
+        self.pool = hs.kv_pool_create(hs.PoolDesc(1, 1, W, Hkv, d, 1, pages))
+        self.sid = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.start = torch.tensor([P], dtype=torch.int64, device=dev)
+        if kind == "swa":
+            kp = gen(synth.TAG_K, 0, self.seq, P - W, W, Hkv, d, 1.0, dev)[None]
+            vp = gen(synth.TAG_V, 0, self.seq, P - W, W, Hkv, d, 1.0, dev)[None]
+            hs.kv_pool_append(self.pool, 0, kp, vp, torch.tensor([P - W], device=dev), seq_ids=self.sid)
+            self.k = gen(synth.TAG_K, 0, self.seq, P, Nc, Hkv, d, 1.0, dev)[None]
+            self.v = gen(synth.TAG_V, 0, self.seq, P, Nc, Hkv, d, 1.0, dev)[None]
+            self.q = gen(synth.TAG_Q, 0, self.seq, P, Nc, Hq, d, 1.0, dev)[None]
+            self.flops = (2 * Nc * Hq * d + 2 * Nc * Hkv * d + 2 * (W - 1) * Hkv * d) * 2  # bytes (metric)
+            self.useful_flops = 4 * d * Nc * W * Hq
+        else:
+            perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 3), pages).to(torch.int32)
+            self.pt = perm.view(1, pages).to(dev)
+            for c0 in range(0, total, 16384):
+                n = min(16384, total - c0)
+                kf = gen(synth.TAG_K, 1, self.seq, c0, n, Hkv, d, 1.0, dev)[None]
+                vf = gen(synth.TAG_V, 1, self.seq, c0, n, Hkv, d, 1.0, dev)[None]
+                hs.kv_pool_append(self.pool, 1, kf, vf, torch.tensor([c0], device=dev), page_table=self.pt)
+            self.q = gen(synth.TAG_Q, 1, self.seq, P, Nc, Hq, d, 1.0, dev)[None]
+            self.flops = 4 * d * (Nc * P + Nc * (Nc + 1) // 2) * Hq
+        self.o = torch.empty_like(self.q)
+        torch.cuda.synchronize()
+
+    def step(self, ev=None):
+        hs = self.hs
+        if ev is not None:
+            ev.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+            ev[-1][0].record()
+        if self.kind == "swa":
+            hs.swa_prefill_fwd(self.pool, 0, self.q, self.k, self.v, o=self.o, start_pos=self.start, seq_ids=self.sid)
+        else:
+            hs.full_prefill_fwd(self.pool, 1, self.q, self.pt, o=self.o, start_pos=self.start)
+        if ev is not None:
+            ev[-1][1].record()
+
+    def e2e_setup(self):
+        self.h_in = [t.cpu().pin_memory() for t in ([self.q, self.k, self.v] if self.kind == "swa" else [self.q])]
+        self.ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(t.numel() * 2 for t in self.h_in)
+        self.d2h = self.ho.numel() * 2
+
+    def e2e_step(self):
+        dev_in = [self.q, self.k, self.v] if self.kind == "swa" else [self.q]
+        for h, d_ in zip(self.h_in, dev_in):
+            d_.copy_(h, non_blocking=True)
+        self.step()
+        self.ho.copy_(self.o, non_blocking=True)
+
+    def _ref_rows(self, rows):
+        P, W, Hkv, d, Hq = self.P, self.W, self.Hkv, self.d, self.Hq
+        if self.kind == "swa":
+            base = P - W + 1
+            k = gen(synth.TAG_K, 0, self.seq, base, self.Nc + W - 1, Hkv, d, 1.0, "cpu")
+            v = gen(synth.TAG_V, 0, self.seq, base, self.Nc + W - 1, Hkv, d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, 0, self.seq, P, self.Nc, Hq, d, 1.0, "cpu")[rows]
+            return q, k, v, W, base
+        k = gen(synth.TAG_K, 1, self.seq, 0, P + self.Nc, Hkv, d, 1.0, "cpu")
+        v = gen(synth.TAG_V, 1, self.seq, 0, P + self.Nc, Hkv, d, 1.0, "cpu")
+        q = gen(synth.TAG_Q, 1, self.seq, P, self.Nc, Hq, d, 1.0, "cpu")[rows]
+        return q, k, v, 0, 0
+
+    def check_sample(self, oracle):
+        rows = [0, 1, 127, 128, 8191, self.Nc - 1] if self.kind == "swa" else [0, 5000, self.Nc - 1]
+        self.step()
+        q, k, v, w, base = self._ref_rows(rows)
+        ref = oracle.attention(q, self.P + np.array(rows), k, v, w, key_base=base)
+        e = np.abs(self.o[0, rows].float().cpu().double().numpy() - ref)
+        return float(e.max()), float(e.mean())
+
+    def oracle_sample(self, oracle, budget_s=10.0, threads=None):
+        """Time the oracle on blocks of rows of this layer until about budget_s; returns
+        (seconds, units of the metric those rows account for, rows)."""
+        rows_all = np.arange(self.Nc)
+        q, k, v, w, base = self._ref_rows(rows_all)
+        done, dt = 0, 0.0
+        block = 512 if self.kind == "swa" else 2
+        while dt < budget_s and done < self.Nc:
+            r = rows_all[done:done + block]
+            t0 = time.perf_counter()
+            oracle.attention(q[r], self.P + r, k, v, w, key_base=base, n_threads=threads)
+            dt += time.perf_counter() - t0
+            done += len(r)
+        if self.kind == "swa":
+            units = self.flops * done / self.Nc
+        else:
+            units = 4 * self.d * self.Hq * sum(self.P + int(i) + 1 for i in rows_all[:done])
+        return dt, units, done
+
+
 class DecodeBatch:
     """Hybrid decode step: n sequences with context lengths log-uniform in [1K, 256K], 4 query
     tokens each (1 + 3 multi-token-prediction drafts), 6 SWA layers on a 128-slot ring and 1 full
@@ -694,7 +803,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", default="hswa", choices=["hswa", "reference"])
     ap.add_argument("--workload", default="swa_prefill_16k",
-                    choices=["swa_prefill_16k", "long_context_1m", "hybrid_decode"])
+                    choices=["swa_prefill_16k", "long_context_1m", "hybrid_decode", "swa_chunk_131k",
+                             "full_chunk_131k"])
     ap.add_argument("--decode-seqs", type=int, default=256, help="sequences in the hybrid_decode batch")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -717,13 +827,20 @@ def main():
     import hybrid_sliding_window_swa_b200 as hs
     hs.load_library()
     hbm, bf16, bf16_sus, peak_src = peaks()
-    decode = args.workload == "hybrid_decode"
-    if big:
+    decode = args.workload in ("hybrid_decode", "swa_chunk_131k")  # bandwidth-bound: GB/s
+    if args.workload in ("swa_chunk_131k", "full_chunk_131k"):
+        wl = HybridChunk131k(hs, kind="swa" if args.workload == "swa_chunk_131k" else "full", seq_offset=rank)
+        dominant_flops = wl.flops
+        if decode:
+            peak, peak_name = hbm, f"{peak_src} HBM copy bandwidth"
+        else:
+            peak, peak_name = bf16, f"{peak_src} bf16 burst"
+    elif big:
         wl = LongContext1M(hs, seq_offset=rank)
         dominant_flops = wl.full_flops_per_launch
         peak = bf16_sus  # a seconds-long step: the sustained figure
         peak_name = f"{peak_src} bf16 sustained"
-    elif decode:
+    elif args.workload == "hybrid_decode":
         wl = DecodeBatch(hs, n=args.decode_seqs, seq_offset=rank)
         wl.flops = wl.bytes  # the decode metric counts bytes
         dominant_flops = wl.full_bytes_per_launch
@@ -796,10 +913,14 @@ def main():
         if not args.no_cpu:
             threads = os.cpu_count() or 1
             dt, fl, nrows = wl.oracle_sample(oracle, threads=threads)
-            if decode:
+            if args.workload == "hybrid_decode":
                 cpu = {"value": fl / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
                        "sample": f"all 4 x 64 rows of the {nrows} shortest sequences on the full layer, fp64, "
                                  f"{dt:.1f} s"}
+            elif args.workload in ("swa_chunk_131k", "full_chunk_131k"):
+                cpu = {"value": fl / dt / (1e9 if decode else 1e12), "unit": "GB/s" if decode else "TFLOP/s",
+                       "cores": threads, "kind": "oracle",
+                       "sample": f"{nrows} query rows x 64 heads of the layer, fp64, {dt:.1f} s"}
             else:
                 what = ("32 heads at the end of sequence 0 (full 4096-key windows)" if not big else
                         "64 heads of SWA layer 3 (full 128-key windows)")
@@ -816,6 +937,14 @@ def main():
                       "l2": "inputs larger than L2 (each full layer reads 4 GiB of pages)",
                       "footprint": wl.footprint()}
             kname = "prefill_kernel<128> (full_prefill_fwd, one full layer)"
+        elif args.workload in ("swa_chunk_131k", "full_chunk_131k"):
+            config = {"workload": wl.name, "B_per_gpu": 1, "prefix": wl.P, "chunk": wl.Nc,
+                      "window": wl.W if wl.kind == "swa" else None, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
+                      "parallelism": f"independent sequences x{ws}",
+                      "step": "swa_prefill_fwd" if wl.kind == "swa" else "full_prefill_fwd (chunk appended first)",
+                      "l2": "inputs larger than L2"}
+            kname = ("prefill_kernel<128> (swa_prefill_fwd)" if wl.kind == "swa" else
+                     "prefill_kernel<128> (full_prefill_fwd)")
         elif decode:
             config = {"workload": wl.name, "n_seqs_per_gpu": wl.n, "sum_ctx": wl.S, "max_ctx": wl.maxL,
                       "tokens_per_seq": wl.nq, "window": wl.W, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
