@@ -903,9 +903,11 @@ def main():
         e2e = {"value": round(wl.flops * ws / e2e_ms / scale, 2), "unit": "GB/s" if decode else "TFLOP/s",
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
                "path": ("pinned host Q and new K/V of 7 layers -> device, 7 hybrid_decode_fwd calls via the Python "
-                        "binding (C ABI), O of 7 layers -> pinned host") if decode else
+                        "binding (C ABI), O of 7 layers -> pinned host") if args.workload == "hybrid_decode" else
                        ("pinned host Q/K/V -> device, swa_prefill_fwd + kv_pool_append via the Python binding "
-                        "(C ABI), O -> pinned host")}
+                        "(C ABI), O -> pinned host") if args.workload == "swa_prefill_16k" else
+                       "pinned host inputs of the chunk -> device, the attention call via the Python binding (C ABI), "
+                       "O -> pinned host"}
     if rank == 0:
         import oracle
         oracle.build()
