@@ -243,6 +243,14 @@ static int build_q_map(CUtensorMap* m, const void* base, int B, int n_q, int H, 
   return make_tmap_bf16(m, base, 4, dims, strides, box) ? HSWA_OK : HSWA_ERR_CUDA;
 }
 
+// Output map: the epilogue of each warp stores its 32 rows of one 64-column half per box.
+static int build_o_map(CUtensorMap* m, void* base, int B, int n_q, int H, int d) {
+  const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)n_q, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)H * d * 2, (uint64_t)n_q * H * d * 2};
+  const uint32_t box[4] = {64, 1, 32, 1};
+  return make_tmap_bf16(m, base, 4, dims, strides, box) ? HSWA_OK : HSWA_ERR_CUDA;
+}
+
 int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k, const hswa_bf16* v,
                     hswa_bf16* o, int B, int n_q, const int64_t* start_pos, const int32_t* seq_ids, int n_q_heads,
                     void* stream) {
@@ -285,6 +293,7 @@ int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_b
   if ((rc = build_q_map(&L.tm_q, q, B, n_q, n_q_heads, D.head_dim))) return rc;
   if ((rc = build_q_map(&L.tm_k, k, B, n_q, D.n_kv_heads, D.head_dim))) return rc;
   if ((rc = build_q_map(&L.tm_v, v, B, n_q, D.n_kv_heads, D.head_dim))) return rc;
+  if ((rc = build_o_map(&L.tm_o, o, B, n_q, n_q_heads, D.head_dim))) return rc;
   return launch_prefill(L, static_cast<cudaStream_t>(stream));
 }
 
@@ -327,6 +336,7 @@ int full_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, hswa_bf16* 
   if ((rc = build_q_map(&L.tm_q, q, B, n_q, n_q_heads, D.head_dim))) return rc;
   L.tm_k = pool->tm_page_k;
   L.tm_v = pool->tm_page_v;
+  if ((rc = build_o_map(&L.tm_o, o, B, n_q, n_q_heads, D.head_dim))) return rc;
   return launch_prefill(L, static_cast<cudaStream_t>(stream));
 }
 

@@ -57,6 +57,7 @@ struct PrefillLaunch {
   int full_layer;      // full layer index within the paged pool (full)
   // tensor maps built by the ABI layer
   CUtensorMap tm_q, tm_k, tm_v;  // tm_k/tm_v: chunk K/V (SWA) or pages (full)
+  CUtensorMap tm_o;              // output, stored 32 rows x 64 columns per TMA box
 };
 
 int launch_prefill(const PrefillLaunch& L, cudaStream_t stream);

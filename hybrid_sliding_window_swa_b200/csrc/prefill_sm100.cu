@@ -18,7 +18,8 @@
 //               row (TMEM lane); all 128 scores of a row in registers, online max/sum
 //               in the exp2 domain with lazy O rescaling, exponentials split between
 //               the MUFU unit and an FMA-pipe polynomial, P written back over S as
-//               packed bf16, and the epilogue (O / l -> bf16 -> global).
+//               packed bf16, and the epilogue (O / l -> bf16, staged in shared memory per
+//               warp and written by TMA stores).
 //   warps 8-11  a third warpgroup that gives its registers to the softmax warpgroups
 //               (setmaxnreg, by default 2 x 128 x 216 + 128 x 72 = the 384 x 168 the CTA launches with):
 //   warp 8      producer: Q of each unit, then K/V tiles into a 2-stage ring of
@@ -100,8 +101,10 @@ struct Layout {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + NQT * TILE;
   static constexpr int V_OFF = K_OFF + NSTAGE * TILE;
-  static constexpr int BAR_OFF = V_OFF + NSTAGE * TILE;
+  static constexpr int O_OFF = V_OFF + NSTAGE * TILE;   // output staging: 4 KB (32 rows x 128 B) per softmax warp
+  static constexpr int BAR_OFF = O_OFF + 2 * BLOCK;
   static constexpr int BYTES = BAR_OFF + 256;
+  static_assert(BYTES + 1024 <= 227 * 1024, "shared memory per CTA");
   static constexpr int O_COL0 = 256;
   static constexpr int O_STRIDE = 128;
 };
@@ -428,7 +431,8 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
 // ---------------------------------------------------------------- softmax + epilogue
 
 template <int D>
-__device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase, const int q) {
+__device__ void softmax_wg(const Params& p, uint8_t* smem, Bars* bars, uint32_t tbase, const int q,
+                           const CUtensorMap* tm_o) {
   using L = Layout<D>;
   const int wq = (threadIdx.x >> 5) & 3;
   const int lane = threadIdx.x & 31;
@@ -658,24 +662,37 @@ __device__ void softmax_wg(const Params& p, Bars* bars, uint32_t tbase, const in
     if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
     ++no;
     tc_fence_after();
-    const int64_t row = (int64_t)qt * BM + r;
-    const bool valid = row < p.n_q;
+    // O / l -> bf16, staged per warp (its 32 rows x 128 B, 128-byte swizzle) and written by one
+    // TMA store per 64-column half; rows past the end of the chunk fall outside the map.
     const float inv = 1.f / l;
-    uint16_t* out = p.o + (((int64_t)G.b * p.n_q + row) * p.Hq + G.h) * D;
+    uint8_t* stage = smem + L::O_OFF + q * L::BLOCK + wq * 4096;
+    const int row0 = qt * BM + wq * 32;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      tmem_ld32(trow + o_col + c0, o);
-      tmem_wait_ld();
-      reg_fence32(o);
-      uint32_t pk[16];
+    for (int dh = 0; dh < D / 64; ++dh) {
+      if (lane == 0) bulk_wait_read_all();  // the previous store from this buffer has read it
+      __syncwarp();
 #pragma unroll
-      for (int k = 0; k < 32; k += 2)
-        pk[k >> 1] = pack_bf16x2(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv);
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(out + c0);
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(trow + o_col + dh * 64 + c0, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        uint32_t pk[16];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        for (int k = 0; k < 32; k += 2)
+          pk[k >> 1] = pack_bf16x2(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int chunk = (c0 >> 3) + x;
+          *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+              make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && row0 < p.n_q) {  // a box wholly past the chunk end is not issued
+        tma_store_4d(tm_o, stage, dh * 64, G.h, row0, G.b);
+        bulk_commit_group();
       }
     }
     // O of this query tile has been read: the next unit's first P V may overwrite it
@@ -688,7 +705,8 @@ template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_rk, const __grid_constant__ CUtensorMap tm_rv) {
+                   const __grid_constant__ CUtensorMap tm_rk, const __grid_constant__ CUtensorMap tm_rv,
+                   const __grid_constant__ CUtensorMap tm_o) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -715,6 +733,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     fence_barrier_init();
   }
   if (warp == PRODUCER_WARP && (threadIdx.x & 31) == 0) {
+    tma_prefetch_desc(&tm_o);
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -731,7 +750,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp < 8) {
     // two softmax warpgroups take the registers the third one gives back
     asm volatile("setmaxnreg.inc.sync.aligned.u32 " HSWA_STR(HSWA_SOFTMAX_REGS) ";" ::: "memory");
-    softmax_wg<D>(p, bars, tbase, warp >> 2);
+    softmax_wg<D>(p, smem, bars, tbase, warp >> 2, &tm_o);
+    if ((threadIdx.x & 31) == 0) bulk_wait_all();  // output stores complete before the CTA exits
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 " HSWA_STR(HSWA_PRODUCER_REGS) ";" ::: "memory");
     if (warp == PRODUCER_WARP) {
@@ -797,11 +817,11 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
   if (Lc.d == 128) {
     const int smem = Layout<128>::BYTES + 1024;
     cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_kernel<128><<<grid, NTHREADS, smem, stream>>>(p, Lc.tm_q, Lc.tm_k, Lc.tm_v, rk, rv);
+    prefill_kernel<128><<<grid, NTHREADS, smem, stream>>>(p, Lc.tm_q, Lc.tm_k, Lc.tm_v, rk, rv, Lc.tm_o);
   } else {
     const int smem = Layout<64>::BYTES + 1024;
     cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_kernel<64><<<grid, NTHREADS, smem, stream>>>(p, Lc.tm_q, Lc.tm_k, Lc.tm_v, rk, rv);
+    prefill_kernel<64><<<grid, NTHREADS, smem, stream>>>(p, Lc.tm_q, Lc.tm_k, Lc.tm_v, rk, rv, Lc.tm_o);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
