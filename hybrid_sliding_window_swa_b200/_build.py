@@ -10,8 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhswa.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["hswa_abi.cu", "pool_kernels.cu", "prefill_sm100.cu", "decode.cu"]
-HEADERS = ["common.cuh", "internal.h"]
+SOURCES = ["hswa_abi.cu", "pool_kernels.cu", "prefill_sm100.cu", "prefill_narrow.cu", "decode.cu"]
+HEADERS = ["common.cuh", "internal.h", "prefill_tile.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -61,6 +61,8 @@ struct PrefillLaunch {
 };
 
 int launch_prefill(const PrefillLaunch& L, cudaStream_t stream);
+// Sliding-window prefill with 1 <= W <= 129 (the band of a query tile spans at most two key tiles).
+int launch_prefill_narrow(const PrefillLaunch& L, cudaStream_t stream);
 
 struct DecodeLaunch {
   int n_seqs, n_qt, Hq, Hkv, d;

@@ -35,43 +35,18 @@
 // absolute positions [128 j, 128 j + 128) = two 64-token pages.
 #include "common.cuh"
 #include "internal.h"
+#include "prefill_tile.cuh"
 
 namespace hswa {
 
 namespace {
 
-constexpr int BM = 128;     // query rows per tile
-constexpr int BN = 128;     // keys per tile
 constexpr int NQT = 2;      // query tiles per unit
 constexpr int NSTAGE = 2;   // K/V pipeline depth
 constexpr int NWARPS = 12;         // 3 warpgroups: registers are granted per warpgroup
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <= 2^8
-
-// Tuning parameters (compile-time):
-//  HSWA_POLY_PER8           pairs of scores in every 8 whose exponential runs on the FMA pipe
-//  HSWA_SOFTMAX_SINGLE_PASS 1: keep all 128 scores of a row in registers (one TMEM read);
-//                           0: read S twice (row maximum, then exponentials), fewer registers
-//  HSWA_SOFTMAX_REGS / HSWA_PRODUCER_REGS  setmaxnreg split (2 * 128 * a + 128 * b <= 384 * 168)
-#ifndef HSWA_POLY_PER8
-#define HSWA_POLY_PER8 0
-#endif
-#ifndef HSWA_SOFTMAX_SINGLE_PASS
-#define HSWA_SOFTMAX_SINGLE_PASS 1
-#endif
-#ifndef HSWA_SOFTMAX_REGS
-#define HSWA_SOFTMAX_REGS 216
-#endif
-#ifndef HSWA_PRODUCER_REGS
-#define HSWA_PRODUCER_REGS 72
-#endif
-static_assert(2 * 128 * HSWA_SOFTMAX_REGS + 128 * HSWA_PRODUCER_REGS <= 384 * 168, "register split");
-#define HSWA_STR2(x) #x
-#define HSWA_STR(x) HSWA_STR2(x)
-
-__device__ __forceinline__ constexpr bool use_poly(int pair) { return (pair & 7) >= 8 - HSWA_POLY_PER8; }
 
 struct Params {
   int B, n_q, Hq, Hkv, G;
@@ -181,12 +156,6 @@ __device__ __forceinline__ bool needs(const Geo& G, int q, int j) {
   return G.act[q] && j >= G.jlo[q] && j <= G.jhi[q];
 }
 
-// All (row, key) pairs of the tile are inside the band.
-__device__ __forceinline__ bool mask_free(const Params& p, const Geo& G, int q, int j) {
-  const int kb = key_base(p, G, j);
-  return kb + BN - 1 <= G.i0[q] && kb >= window_lo(p, G.i1[q]);
-}
-
 // ---------------------------------------------------------------- producer
 
 // Rolling-buffer rows of one key tile with cp.async (general W and chunk start):
@@ -199,21 +168,7 @@ __device__ __forceinline__ void ring_tile_cpasync(const Params& p, const Geo& G,
   if (!seq_ok && lane == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
   const int64_t row_base = seq_ok ? (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + G.g) * p.window : 0;
   const int held_lo = (G.P - p.window > 0) ? G.P - p.window : 0;
-  const uint32_t sdst = smem_u32(dst);
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  for (int idx = lane; idx < BN * CH; idx += 32) {
-    const int r = idx / CH;
-    const int c = idx % CH;
-    const int pos = kb + r;
-    const bool held = seq_ok && pos >= held_lo && pos < G.P;
-    const uint16_t* src = ring + (held ? (row_base + (pos % p.window)) * D + c * 8 : 0);
-    const int blk = c >> 3, cc = c & 7;
-    const uint32_t off = blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
-    cp_async_16(sdst + off, src, held ? 16u : 0u);
-  }
-  cp_async_wait_all();
-  fence_proxy_async_smem();
-  __syncwarp();
+  ring_rows_cpasync<D>(ring + row_base * D, seq_ok, held_lo, G.P, p.window, dst, kb, lane);
 }
 
 template <int D>
@@ -471,188 +426,7 @@ __device__ void softmax_wg(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
       const bool edge = !(kb + BN - 1 <= qi0 && kb >= lo_last);
       const int c_lo = lo_i - kb;
       const int c_hi = i - kb;
-#if HSWA_SOFTMAX_SINGLE_PASS
-      // all 128 scores of the row: four TMEM loads, one wait
-      uint32_t v[128];
-      tmem_ld32_into<0>(trow + s_col + 0, v);
-      tmem_ld32_into<32>(trow + s_col + 32, v);
-      tmem_ld32_into<64>(trow + s_col + 64, v);
-      tmem_ld32_into<96>(trow + s_col + 96, v);
-      tmem_wait_ld();
-      reg_fence_into<0>(v);
-      reg_fence_into<32>(v);
-      reg_fence_into<64>(v);
-      reg_fence_into<96>(v);
-      if (edge) {
-#pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (k < c_lo || k > c_hi) v[k] = __float_as_uint(-INFINITY);
-      }
-      float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
-      float m2 = __uint_as_float(v[2]), m3 = __uint_as_float(v[3]);
-#pragma unroll
-      for (int k = 4; k < 124; k += 8) {
-        m0 = fmax3(m0, __uint_as_float(v[k + 0]), __uint_as_float(v[k + 1]));
-        m1 = fmax3(m1, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
-        m2 = fmax3(m2, __uint_as_float(v[k + 4]), __uint_as_float(v[k + 5]));
-        m3 = fmax3(m3, __uint_as_float(v[k + 6]), __uint_as_float(v[k + 7]));
-      }
-      m0 = fmax3(m0, __uint_as_float(v[124]), __uint_as_float(v[125]));
-      m1 = fmax3(m1, __uint_as_float(v[126]), __uint_as_float(v[127]));
-      const float mx = fmaxf(fmax3(m0, m1, m2), m3);
-      const float m_tile = mx * sl2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_tile > m_used + kTau) {
-        if (m_used != -INFINITY) {
-          alpha = ex2_approx(m_used - m_tile);
-          resc = true;
-        }
-        l *= alpha;
-        m_used = m_tile;
-      }
-      if (__any_sync(0xffffffffu, resc) && n_done > 0) {
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(trow + o_col + c0, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(trow + o_col + c0, o);
-        }
-        tmem_wait_st();
-      }
-      // P = 2^(s * scale * log2 e - m) in place, packed to bf16 and stored over S
-      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
-      const uint64_t scale2 = f2_pack(sl2, sl2);
-      const uint64_t neg2 = f2_pack(-moff, -moff);
-      uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const int pair = (c0 + k) >> 1;
-          const uint64_t x = f2_fma(f2_pack(__uint_as_float(v[c0 + k]), __uint_as_float(v[c0 + k + 1])), scale2, neg2);
-          uint64_t e;
-          if (use_poly(pair)) {
-            e = exp2_poly_x2(x);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          }
-          acc[pair & 3] = f2_add(acc[pair & 3], e);
-          float e0, e1;
-          f2_unpack(e, e0, e1);
-          pk[k >> 1] = pack_bf16x2(e0, e1);
-        }
-        tmem_st16(trow + s_col + (c0 >> 1), pk);
-      }
-#else
-      // pass 1: row maximum, 64 scores at a time
-      float mx = -INFINITY;
-#pragma unroll
-      for (int h2 = 0; h2 < BN; h2 += 64) {
-        uint32_t va[32], vb[32];
-        tmem_ld32(trow + s_col + h2, va);
-        tmem_ld32(trow + s_col + h2 + 32, vb);
-        tmem_wait_ld();
-        reg_fence32(va);
-        reg_fence32(vb);
-        if (edge) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (h2 + k < c_lo || h2 + k > c_hi) va[k] = __float_as_uint(-INFINITY);
-            if (h2 + 32 + k < c_lo || h2 + 32 + k > c_hi) vb[k] = __float_as_uint(-INFINITY);
-          }
-        }
-        float m0 = mx, m1 = __uint_as_float(va[0]), m2 = __uint_as_float(vb[0]);
-#pragma unroll
-        for (int k = 1; k < 31; k += 2) {
-          m0 = fmax3(m0, __uint_as_float(va[k]), __uint_as_float(va[k + 1]));
-          m1 = fmax3(m1, __uint_as_float(vb[k]), __uint_as_float(vb[k + 1]));
-        }
-        m2 = fmax3(m2, __uint_as_float(va[31]), __uint_as_float(vb[31]));
-        mx = fmax3(m0, m1, m2);
-      }
-      const float m_tile = mx * sl2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_tile > m_used + kTau) {
-        if (m_used != -INFINITY) {
-          alpha = ex2_approx(m_used - m_tile);
-          resc = true;
-        }
-        l *= alpha;
-        m_used = m_tile;
-      }
-      if (__any_sync(0xffffffffu, resc) && n_done > 0) {
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(trow + o_col + c0, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(trow + o_col + c0, o);
-        }
-        tmem_wait_st();
-      }
-      // pass 2: P = 2^(s * scale * log2 e - m), 32 columns at a time, the next chunk's TMEM
-      // load in flight while this one is exponentiated, packed and stored over S.
-      const float moff = (m_used == -INFINITY) ? 0.f : m_used;
-      const uint64_t scale2 = f2_pack(sl2, sl2);
-      const uint64_t neg2 = f2_pack(-moff, -moff);
-      uint64_t acc[4] = {0, 0, 0, 0};
-      uint32_t buf[2][32];
-      tmem_ld32(trow + s_col, buf[0]);
-      tmem_wait_ld();
-      reg_fence32(buf[0]);
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t(&cur)[32] = buf[c & 1];
-        if (c + 1 < BN / 32) tmem_ld32(trow + s_col + 32 * (c + 1), buf[(c + 1) & 1]);
-        const int c0 = 32 * c;
-        if (edge) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (c0 + k < c_lo || c0 + k > c_hi) cur[k] = __float_as_uint(-INFINITY);
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const int pair = (c0 + k) >> 1;
-          const uint64_t x = f2_fma(f2_pack(__uint_as_float(cur[k]), __uint_as_float(cur[k + 1])), scale2, neg2);
-          uint64_t e;
-          if (use_poly(pair)) {
-            e = exp2_poly_x2(x);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            e = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          }
-          acc[pair & 3] = f2_add(acc[pair & 3], e);
-          float e0, e1;
-          f2_unpack(e, e0, e1);
-          pk[k >> 1] = pack_bf16x2(e0, e1);
-        }
-        tmem_st16(trow + s_col + (c0 >> 1), pk);
-        if (c + 1 < BN / 32) {
-          tmem_wait_ld();
-          reg_fence32(buf[(c + 1) & 1]);
-        }
-      }
-#endif
-      float a0, a1, b0, b1, c0_, c1_, d0, d1;
-      f2_unpack(acc[0], a0, a1);
-      f2_unpack(acc[1], b0, b1);
-      f2_unpack(acc[2], c0_, c1_);
-      f2_unpack(acc[3], d0, d1);
-      l += ((a0 + a1) + (b0 + b1)) + ((c0_ + c1_) + (d0 + d1));
+      softmax_tile<D>(trow, s_col, o_col, sl2, edge, c_lo, c_hi, m_used, l, n_done > 0);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[q]);
@@ -662,39 +436,8 @@ __device__ void softmax_wg(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
     if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
     ++no;
     tc_fence_after();
-    // O / l -> bf16, staged per warp (its 32 rows x 128 B, 128-byte swizzle) and written by one
-    // TMA store per 64-column half; rows past the end of the chunk fall outside the map.
-    const float inv = 1.f / l;
-    uint8_t* stage = smem + L::O_OFF + q * L::BLOCK + wq * 4096;
-    const int row0 = qt * BM + wq * 32;
-#pragma unroll
-    for (int dh = 0; dh < D / 64; ++dh) {
-      if (lane == 0) bulk_wait_read_all();  // the previous store from this buffer has read it
-      __syncwarp();
-#pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(trow + o_col + dh * 64 + c0, o);
-        tmem_wait_ld();
-        reg_fence32(o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2)
-          pk[k >> 1] = pack_bf16x2(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int chunk = (c0 >> 3) + x;
-          *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-              make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && row0 < p.n_q) {  // a box wholly past the chunk end is not issued
-        tma_store_4d(tm_o, stage, dh * 64, G.h, row0, G.b);
-        bulk_commit_group();
-      }
-    }
+    store_output<D>(trow, o_col, l, smem + L::O_OFF + q * L::BLOCK + wq * 4096, lane, tm_o, G.h, qt * BM + wq * 32,
+                    G.b, p.n_q);
     // O of this query tile has been read: the next unit's first P V may overwrite it
     // (ordered by this warpgroup's next p_full arrival).
     tc_fence_before();
@@ -773,6 +516,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace
 
 int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
+  // narrow windows: every query tile's band fits in two key tiles, which stay resident while
+  // all query heads of a KV head pass through them
+  if (Lc.window >= 1 && Lc.window <= BN + 1) return launch_prefill_narrow(Lc, stream);
   const hswa_pool* pool = Lc.pool;
   const hswa_pool_desc& D = pool->desc;
   Params p{};

@@ -1,0 +1,296 @@
+// prefill_tile.cuh -- per-tile pieces shared by the prefill kernels: the online-softmax step of
+// one 128-key tile for one query row (one thread per TMEM lane), the output epilogue, and the
+// cp.async loader for rolling-buffer rows.
+//
+// Math ("Sliding Window Attention (SWA) no riron to jisso", section "formal definition",
+// eqs. (1)-(5)): row i's weights are softmax_j(q_i . k_j / sqrt(d)) over the keys of its band;
+// the step keeps the running maximum in the exp2 domain and rescales O only when the maximum
+// grows by more than 2^kTau, so P = 2^(s * scale * log2 e - m) stays below 2^kTau.
+#pragma once
+#include "common.cuh"
+
+namespace hswa {
+namespace {
+
+constexpr int BM = 128;     // query rows per tile
+constexpr int BN = 128;     // keys per tile
+constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <= 2^8
+
+// Tuning parameters (compile-time):
+//  HSWA_POLY_PER8           pairs of scores in every 8 whose exponential runs on the FMA pipe
+//  HSWA_SOFTMAX_SINGLE_PASS 1: keep all 128 scores of a row in registers (one TMEM read);
+//                           0: read S twice (row maximum, then exponentials), fewer registers
+//  HSWA_SOFTMAX_REGS / HSWA_PRODUCER_REGS  setmaxnreg split (2 * 128 * a + 128 * b <= 384 * 168)
+#ifndef HSWA_POLY_PER8
+#define HSWA_POLY_PER8 0
+#endif
+#ifndef HSWA_SOFTMAX_SINGLE_PASS
+#define HSWA_SOFTMAX_SINGLE_PASS 1
+#endif
+#ifndef HSWA_SOFTMAX_REGS
+#define HSWA_SOFTMAX_REGS 216
+#endif
+#ifndef HSWA_PRODUCER_REGS
+#define HSWA_PRODUCER_REGS 72
+#endif
+static_assert(2 * 128 * HSWA_SOFTMAX_REGS + 128 * HSWA_PRODUCER_REGS <= 384 * 168, "register split");
+#define HSWA_STR2(x) #x
+#define HSWA_STR(x) HSWA_STR2(x)
+
+__device__ __forceinline__ constexpr bool use_poly(int pair) { return (pair & 7) >= 8 - HSWA_POLY_PER8; }
+
+// One key tile of one query row. trow: this warp's TMEM lane base; S of the row in columns
+// [s_col, s_col + 128), O in [o_col, o_col + D). Columns outside [c_lo, c_hi] are masked when
+// `edge`. m_used / l: running maximum (log2 domain) and row sum; o_live: O already holds a
+// partial sum (it is rescaled when the maximum moves). P is written over S as packed bf16;
+// the caller waits for the TMEM stores and signals the MMA.
+template <int D>
+__device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint32_t o_col, float sl2, bool edge,
+                                             int c_lo, int c_hi, float& m_used, float& l, bool o_live) {
+#if HSWA_SOFTMAX_SINGLE_PASS
+    // all 128 scores of the row: four TMEM loads, one wait
+    uint32_t v[128];
+    tmem_ld32_into<0>(trow + s_col + 0, v);
+    tmem_ld32_into<32>(trow + s_col + 32, v);
+    tmem_ld32_into<64>(trow + s_col + 64, v);
+    tmem_ld32_into<96>(trow + s_col + 96, v);
+    tmem_wait_ld();
+    reg_fence_into<0>(v);
+    reg_fence_into<32>(v);
+    reg_fence_into<64>(v);
+    reg_fence_into<96>(v);
+    if (edge) {
+#pragma unroll
+      for (int k = 0; k < 128; ++k)
+        if (k < c_lo || k > c_hi) v[k] = __float_as_uint(-INFINITY);
+    }
+    float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
+    float m2 = __uint_as_float(v[2]), m3 = __uint_as_float(v[3]);
+#pragma unroll
+    for (int k = 4; k < 124; k += 8) {
+      m0 = fmax3(m0, __uint_as_float(v[k + 0]), __uint_as_float(v[k + 1]));
+      m1 = fmax3(m1, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+      m2 = fmax3(m2, __uint_as_float(v[k + 4]), __uint_as_float(v[k + 5]));
+      m3 = fmax3(m3, __uint_as_float(v[k + 6]), __uint_as_float(v[k + 7]));
+    }
+    m0 = fmax3(m0, __uint_as_float(v[124]), __uint_as_float(v[125]));
+    m1 = fmax3(m1, __uint_as_float(v[126]), __uint_as_float(v[127]));
+    const float mx = fmaxf(fmax3(m0, m1, m2), m3);
+    const float m_tile = mx * sl2;
+    float alpha = 1.f;
+    bool resc = false;
+    if (m_tile > m_used + kTau) {
+      if (m_used != -INFINITY) {
+        alpha = ex2_approx(m_used - m_tile);
+        resc = true;
+      }
+      l *= alpha;
+      m_used = m_tile;
+    }
+    if (__any_sync(0xffffffffu, resc) && o_live) {
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(trow + o_col + c0, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+        tmem_st32(trow + o_col + c0, o);
+      }
+      tmem_wait_st();
+    }
+    // P = 2^(s * scale * log2 e - m) in place, packed to bf16 and stored over S
+    const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+    const uint64_t scale2 = f2_pack(sl2, sl2);
+    const uint64_t neg2 = f2_pack(-moff, -moff);
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        const int pair = (c0 + k) >> 1;
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(v[c0 + k]), __uint_as_float(v[c0 + k + 1])), scale2, neg2);
+        uint64_t e;
+        if (use_poly(pair)) {
+          e = exp2_poly_x2(x);
+        } else {
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        acc[pair & 3] = f2_add(acc[pair & 3], e);
+        float e0, e1;
+        f2_unpack(e, e0, e1);
+        pk[k >> 1] = pack_bf16x2(e0, e1);
+      }
+      tmem_st16(trow + s_col + (c0 >> 1), pk);
+    }
+#else
+    // pass 1: row maximum, 64 scores at a time
+    float mx = -INFINITY;
+#pragma unroll
+    for (int h2 = 0; h2 < BN; h2 += 64) {
+      uint32_t va[32], vb[32];
+      tmem_ld32(trow + s_col + h2, va);
+      tmem_ld32(trow + s_col + h2 + 32, vb);
+      tmem_wait_ld();
+      reg_fence32(va);
+      reg_fence32(vb);
+      if (edge) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          if (h2 + k < c_lo || h2 + k > c_hi) va[k] = __float_as_uint(-INFINITY);
+          if (h2 + 32 + k < c_lo || h2 + 32 + k > c_hi) vb[k] = __float_as_uint(-INFINITY);
+        }
+      }
+      float m0 = mx, m1 = __uint_as_float(va[0]), m2 = __uint_as_float(vb[0]);
+#pragma unroll
+      for (int k = 1; k < 31; k += 2) {
+        m0 = fmax3(m0, __uint_as_float(va[k]), __uint_as_float(va[k + 1]));
+        m1 = fmax3(m1, __uint_as_float(vb[k]), __uint_as_float(vb[k + 1]));
+      }
+      m2 = fmax3(m2, __uint_as_float(va[31]), __uint_as_float(vb[31]));
+      mx = fmax3(m0, m1, m2);
+    }
+    const float m_tile = mx * sl2;
+    float alpha = 1.f;
+    bool resc = false;
+    if (m_tile > m_used + kTau) {
+      if (m_used != -INFINITY) {
+        alpha = ex2_approx(m_used - m_tile);
+        resc = true;
+      }
+      l *= alpha;
+      m_used = m_tile;
+    }
+    if (__any_sync(0xffffffffu, resc) && o_live) {
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(trow + o_col + c0, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+        tmem_st32(trow + o_col + c0, o);
+      }
+      tmem_wait_st();
+    }
+    // pass 2: P = 2^(s * scale * log2 e - m), 32 columns at a time, the next chunk's TMEM
+    // load in flight while this one is exponentiated, packed and stored over S.
+    const float moff = (m_used == -INFINITY) ? 0.f : m_used;
+    const uint64_t scale2 = f2_pack(sl2, sl2);
+    const uint64_t neg2 = f2_pack(-moff, -moff);
+    uint64_t acc[4] = {0, 0, 0, 0};
+    uint32_t buf[2][32];
+    tmem_ld32(trow + s_col, buf[0]);
+    tmem_wait_ld();
+    reg_fence32(buf[0]);
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t(&cur)[32] = buf[c & 1];
+      if (c + 1 < BN / 32) tmem_ld32(trow + s_col + 32 * (c + 1), buf[(c + 1) & 1]);
+      const int c0 = 32 * c;
+      if (edge) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (c0 + k < c_lo || c0 + k > c_hi) cur[k] = __float_as_uint(-INFINITY);
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        const int pair = (c0 + k) >> 1;
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(cur[k]), __uint_as_float(cur[k + 1])), scale2, neg2);
+        uint64_t e;
+        if (use_poly(pair)) {
+          e = exp2_poly_x2(x);
+        } else {
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        acc[pair & 3] = f2_add(acc[pair & 3], e);
+        float e0, e1;
+        f2_unpack(e, e0, e1);
+        pk[k >> 1] = pack_bf16x2(e0, e1);
+      }
+      tmem_st16(trow + s_col + (c0 >> 1), pk);
+      if (c + 1 < BN / 32) {
+        tmem_wait_ld();
+        reg_fence32(buf[(c + 1) & 1]);
+      }
+    }
+#endif
+    float a0, a1, b0, b1, c0_, c1_, d0, d1;
+    f2_unpack(acc[0], a0, a1);
+    f2_unpack(acc[1], b0, b1);
+    f2_unpack(acc[2], c0_, c1_);
+    f2_unpack(acc[3], d0, d1);
+    l += ((a0 + a1) + (b0 + b1)) + ((c0_ + c1_) + (d0 + d1));
+}
+
+// Epilogue of one query tile: O / l -> bf16, staged per warp (its 32 rows x 128 B, 128-byte
+// swizzle, 4 KB at `stage`) and written by one TMA store per 64-column half into the output
+// map at (column, head h, row0 .. row0 + 31, batch b); rows past n_q fall outside the map.
+template <int D>
+__device__ __forceinline__ void store_output(uint32_t trow, uint32_t o_col, float l, uint8_t* stage, int lane,
+                                             const CUtensorMap* tm_o, int h, int row0, int b, int n_q) {
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int dh = 0; dh < D / 64; ++dh) {
+    if (lane == 0) bulk_wait_read_all();  // the previous store from this buffer has read it
+    __syncwarp();
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld32(trow + o_col + dh * 64 + c0, o);
+      tmem_wait_ld();
+      reg_fence32(o);
+      uint32_t pk[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2)
+        pk[k >> 1] = pack_bf16x2(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int chunk = (c0 >> 3) + x;
+        *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+            make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row0 < n_q) {  // a box wholly past the chunk end is not issued
+      tma_store_4d(tm_o, stage, dh * 64, h, row0, b);
+      bulk_commit_group();
+    }
+  }
+}
+
+// Rolling-buffer rows of one key tile with cp.async (any W and chunk start), one warp:
+// positions kb .. kb + 127 come from slot pos mod W of the ring at `ring_rows` (W rows of d),
+// rows whose position the ring does not hold ([held_lo, held_hi) holds) or a bad ring are
+// zero-filled. Layout of dst: [D / 64 blocks][128 rows][128 B], 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ void ring_rows_cpasync(const uint16_t* ring_rows, bool ok, int held_lo, int held_hi,
+                                                  int W, uint8_t* dst, int kb, int lane) {
+  const uint32_t sdst = smem_u32(dst);
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  for (int idx = lane; idx < BN * CH; idx += 32) {
+    const int r = idx / CH;
+    const int c = idx % CH;
+    const int pos = kb + r;
+    const bool held = ok && pos >= held_lo && pos < held_hi;
+    const uint16_t* src = held ? ring_rows + (int64_t)(pos % W) * D + c * 8 : ring_rows;
+    const int blk = c >> 3, cc = c & 7;
+    const uint32_t off = blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
+    cp_async_16(sdst + off, src, held ? 16u : 0u);
+  }
+  cp_async_wait_all();
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+
+}  // namespace
+}  // namespace hswa
