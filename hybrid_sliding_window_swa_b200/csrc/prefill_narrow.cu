@@ -10,14 +10,16 @@
 // Work unit = (query tile t, batch row b, KV head g). The band of tile t covers key tiles
 // t - 1 and t (relative to the chunk start; tile -1 is the rolling buffer). Both key tiles
 // are loaded once per unit and stay in shared memory while the G query heads of KV head g
-// stream through two independent slots: slot q takes heads g*G + q, g*G + q + 2, ...
+// stream through two slots: slot q takes heads g*G + q, g*G + q + 2, ...
 //   warps 0-3 / 4-7  softmax + epilogue of slot 0 / slot 1 (one thread per TMEM lane)
 //   warp 8           K/V producer (TMA for chunk rows and aligned ring tiles, cp.async for
 //                    the others)
-//   warp 9, warp 11  MMA issuer of slot 0 / slot 1 (one thread each; warp 9 also owns TMEM)
+//   warp 9           MMA issuer for both slots in a fixed alternating order (one thread; the
+//                    two softmax warpgroups then take turns with the tensor core); owns TMEM
 //   warp 10          Q producer: the next head of a slot is loaded as soon as that slot's last
 //                    S MMA of the current head has read its Q tile, so the load overlaps the
-//                    slot's last softmax, P V and epilogue.
+//                    slot's last softmax, P V and epilogue
+//   warp 11          completes the warpgroup
 // TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D); P is written over S.
 // Shared memory: Q 2 tiles, K 2 tiles, V 2 tiles, output staging 2 x 16 KB.
 #include "common.cuh"
@@ -33,9 +35,8 @@ constexpr int NKT = 2;            // key tiles per unit (at most)
 constexpr int NWARPS = 12;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int KV_WARP = 8;
-constexpr int MMA0_WARP = 9;
+constexpr int MMA_WARP = 9;
 constexpr int QP_WARP = 10;
-constexpr int MMA1_WARP = 11;
 
 struct NParams {
   int B, n_q, Hq, Hkv, G;
@@ -190,74 +191,87 @@ __device__ void q_producer(const NParams& p, uint8_t* smem, NBars* bars, const C
   }
 }
 
-// ---------------------------------------------------------------- MMA issuer (one per slot)
+// ---------------------------------------------------------------- MMA issuer (both slots)
 
+// One thread issues both slots' MMAs in a fixed alternating order, step by step (a step is one
+// key tile of the slots' current heads): O_q += P_q V of the slot's previous S, then the slot's
+// next S. While one slot's softmax runs, the tensor core works on the other slot's products.
 template <int D>
-__device__ void mma_slot(const NParams& p, uint8_t* smem, NBars* bars, uint32_t tbase, const int q) {
+__device__ void mma_issuer(const NParams& p, uint8_t* smem, NBars* bars, uint32_t tbase) {
   using L = NLayout<D>;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
-  const uint32_t q_base = smem_u32(smem + L::Q_OFF + q * L::TILE);
+  const uint32_t q_base = smem_u32(smem + L::Q_OFF);
   const uint32_t k_base = smem_u32(smem + L::K_OFF);
   const uint32_t v_base = smem_u32(smem + L::V_OFF);
-  const uint32_t s_tmem = tbase + q * 128;
-  const uint32_t o_tmem = tbase + L::O_COL0 + q * 128;
-  uint32_t np = 0;     // P tiles consumed (p_full phase)
-  uint32_t nqf = 0;    // Q tiles consumed (q_full phase)
-  uint32_t kvph = 0;   // bit jj: kv_full phase of key-tile slot jj
-
-  auto issue_s = [&](int jj) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * L::BLOCK + (kk & 3) * 32;
-      const uint64_t adesc = smem_desc_sw128(q_base + off, 16, 1024);
-      const uint64_t bdesc = smem_desc_sw128(k_base + jj * L::TILE + off, 16, 1024);
-      umma_ss(s_tmem, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
-    }
-    umma_commit(&bars->s_full[q]);
-  };
-  // O (+)= P V of key tile jj, once the softmax has written P
-  auto issue_pv = [&](int jj, bool accumulate) -> bool {
-    if (!mbar_wait(&bars->p_full[q], np & 1, p.err)) return false;
-    ++np;
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-      const uint64_t bdesc = smem_desc_sw128(v_base + jj * L::TILE + kk * 16 * 128, L::BLOCK, 1024);
-      umma_ts(o_tmem, s_tmem + kk * 8, bdesc, IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
-    }
-    return true;
-  };
+  uint32_t np = 0;    // bit q: p_full phase of slot q
+  uint32_t nqf = 0;   // bit q: q_full phase of slot q
+  uint32_t kvph = 0;  // bit jj: kv_full phase of key-tile slot jj
 
   for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
     NGeo G;
     make_ngeo(p, unit, G);
     uint32_t kv_ready = 0;  // bit jj: key tile jj of this unit has landed
-    auto wait_kv = [&](int jj) -> bool {
-      if ((kv_ready >> jj) & 1u) return true;
-      if (!mbar_wait(&bars->kv_full[jj], (kvph >> jj) & 1u, p.err)) return false;
+    int pend_jj[NSLOT] = {-1, -1};  // key tile of a slot's S whose P V is not issued yet
+    bool pend_last[NSLOT] = {false, false};  // ... and it is the head's last key tile
+    auto drain = [&](int q) -> bool {
+      if (pend_jj[q] < 0) return true;
+      if (!mbar_wait(&bars->p_full[q], (np >> q) & 1u, p.err)) return false;
+      np ^= 1u << q;
       tc_fence_after();
-      kv_ready |= 1u << jj;
+      const int jj = pend_jj[q];
+      const uint32_t vb = v_base + jj * L::TILE;
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        const uint64_t bdesc = smem_desc_sw128(vb + kk * 16 * 128, L::BLOCK, 1024);
+        umma_ts(tbase + L::O_COL0 + q * 128, tbase + q * 128 + kk * 8, bdesc, IDESC_PV,
+                (jj > 0 || kk > 0) ? 1u : 0u);
+      }
+      if (pend_last[q]) umma_commit(&bars->o_full[q]);
+      pend_jj[q] = -1;
       return true;
     };
-    for (int k = 0; k < G.nh[q]; ++k) {
-      if (!mbar_wait(&bars->q_full[q], nqf & 1, p.err)) return;
-      ++nqf;
-      tc_fence_after();
+    const int nk = G.nh[0] > G.nh[1] ? G.nh[0] : G.nh[1];
+    for (int k = 0; k < nk; ++k) {
       for (int jj = 0; jj < G.nkt; ++jj) {
-        if (!wait_kv(jj)) return;
-        // P of the previous key tile lives in the S columns: its P V goes first
-        if (jj > 0 && !issue_pv(jj - 1, jj - 1 > 0)) return;
-        issue_s(jj);
-        if (jj == G.nkt - 1) umma_commit(&bars->q_empty[q]);  // this head's Q tile is read
+        if (!((kv_ready >> jj) & 1u)) {
+          if (!mbar_wait(&bars->kv_full[jj], (kvph >> jj) & 1u, p.err)) return;
+          tc_fence_after();
+          kv_ready |= 1u << jj;
+        }
+#pragma unroll
+        for (int q = 0; q < NSLOT; ++q) {
+          // P of the slot's previous key tile lives in its S columns: that P V goes first
+          if (!drain(q)) return;
+          if (k >= G.nh[q]) continue;
+          if (jj == 0) {  // a new head of the slot: its Q tile
+            if (!mbar_wait(&bars->q_full[q], (nqf >> q) & 1u, p.err)) return;
+            nqf ^= 1u << q;
+            tc_fence_after();
+          }
+          const uint32_t qb = q_base + q * L::TILE, kb = k_base + jj * L::TILE;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::BLOCK + (kk & 3) * 32;
+            umma_ss(tbase + q * 128, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                    IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full[q]);
+          if (jj == G.nkt - 1) umma_commit(&bars->q_empty[q]);  // this head's Q tile is read
+          pend_jj[q] = jj;
+          pend_last[q] = jj == G.nkt - 1;
+        }
       }
-      if (!issue_pv(G.nkt - 1, G.nkt > 1)) return;
-      umma_commit(&bars->o_full[q]);
     }
-    // the unit's key tiles are free once both slots' MMAs on them have completed; each slot
-    // waits for a tile before releasing it, so neither releases a phase twice
+    // the last products read the unit's V tiles: issue them, then release the key tiles
+#pragma unroll
+    for (int q = 0; q < NSLOT; ++q)
+      if (!drain(q)) return;
     for (int jj = 0; jj < G.nkt; ++jj) {
-      if (!wait_kv(jj)) return;
+      if (!((kv_ready >> jj) & 1u)) {  // a unit without heads still pairs its waits and releases
+        if (!mbar_wait(&bars->kv_full[jj], (kvph >> jj) & 1u, p.err)) return;
+        tc_fence_after();
+      }
       umma_commit(&bars->kv_empty[jj]);
       kvph ^= 1u << jj;
     }
@@ -336,7 +350,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int jj = 0; jj < NKT; ++jj) {
       mbar_init(&bars->kv_full[jj], 1);
-      mbar_init(&bars->kv_empty[jj], NSLOT);  // one release per slot's MMA issuer
+      mbar_init(&bars->kv_empty[jj], 1);
     }
     fence_barrier_init();
   }
@@ -346,7 +360,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_o);
   }
-  if (warp == MMA0_WARP) {
+  if (warp == MMA_WARP) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -364,8 +378,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == KV_WARP) {
       kv_producer<D>(p, smem, bars, &tm_k, &tm_v, &tm_rk, &tm_rv);
     } else if ((threadIdx.x & 31) == 0) {
-      if (warp == MMA0_WARP) mma_slot<D>(p, smem, bars, tbase, 0);
-      else if (warp == MMA1_WARP) mma_slot<D>(p, smem, bars, tbase, 1);
+      if (warp == MMA_WARP) mma_issuer<D>(p, smem, bars, tbase);
       else if (warp == QP_WARP) q_producer<D>(p, smem, bars, &tm_q);
     }
     __syncwarp();
@@ -373,7 +386,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == MMA0_WARP) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
