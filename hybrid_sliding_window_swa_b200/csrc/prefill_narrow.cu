@@ -261,20 +261,20 @@ __device__ void mma_issuer(const NParams& p, uint8_t* smem, NBars* bars, uint32_
           pend_jj[q] = jj;
           pend_last[q] = jj == G.nkt - 1;
         }
+        // the last products on key tile jj - 1 have just been issued: the producer may refill it
+        // for the next unit while this step's work runs
+        if (k == nk - 1 && jj > 0) {
+          umma_commit(&bars->kv_empty[jj - 1]);
+          kvph ^= 1u << (jj - 1);
+        }
       }
     }
-    // the last products read the unit's V tiles: issue them, then release the key tiles
+    // the last products read the unit's last V tile: issue them, then release that tile
 #pragma unroll
     for (int q = 0; q < NSLOT; ++q)
       if (!drain(q)) return;
-    for (int jj = 0; jj < G.nkt; ++jj) {
-      if (!((kv_ready >> jj) & 1u)) {  // a unit without heads still pairs its waits and releases
-        if (!mbar_wait(&bars->kv_full[jj], (kvph >> jj) & 1u, p.err)) return;
-        tc_fence_after();
-      }
-      umma_commit(&bars->kv_empty[jj]);
-      kvph ^= 1u << jj;
-    }
+    umma_commit(&bars->kv_empty[G.nkt - 1]);
+    kvph ^= 1u << (G.nkt - 1);
   }
 }
 
