@@ -945,7 +945,7 @@ def main():
                       "parallelism": f"independent sequences x{ws}",
                       "step": "swa_prefill_fwd" if wl.kind == "swa" else "full_prefill_fwd (chunk appended first)",
                       "l2": "inputs larger than L2"}
-            kname = ("prefill_kernel<128> (swa_prefill_fwd)" if wl.kind == "swa" else
+            kname = ("prefill_narrow_kernel<128> (swa_prefill_fwd, W <= 129 path)" if wl.kind == "swa" else
                      "prefill_kernel<128> (full_prefill_fwd)")
         elif decode:
             config = {"workload": wl.name, "n_seqs_per_gpu": wl.n, "sum_ctx": wl.S, "max_ctx": wl.maxL,
