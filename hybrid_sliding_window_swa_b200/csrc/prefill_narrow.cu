@@ -311,7 +311,7 @@ __device__ void softmax_slot(const NParams& p, uint8_t* smem, NBars* bars, uint3
         // columns of this row inside the band: [c_lo, c_hi] (edge tiles only)
         const int kb = G.P + BN * (G.jlo + jj);
         const bool edge = !(kb + BN - 1 <= G.i0 && kb >= lo_last);
-        softmax_tile<D>(trow, s_col, o_col, sl2, edge, lo_i - kb, i - kb, m_used, l, jj > 0);
+        softmax_tile<D, false>(trow, s_col, o_col, sl2, edge, lo_i - kb, i - kb, m_used, l, jj > 0);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_full[q]);

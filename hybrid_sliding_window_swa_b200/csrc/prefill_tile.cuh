@@ -44,7 +44,10 @@ __device__ __forceinline__ constexpr bool use_poly(int pair) { return (pair & 7)
 // `edge`. m_used / l: running maximum (log2 domain) and row sum; o_live: O already holds a
 // partial sum (it is rescaled when the maximum moves). P is written over S as packed bf16;
 // the caller waits for the TMEM stores and signals the MMA.
-template <int D>
+// BRANCH_FREE_MASK selects how edge tiles are masked: integer sign arithmetic on every column
+// (faster where edge tiles are few, as in long windows) or per-column compares (faster where
+// every tile is an edge tile, as in the narrow-window kernel); both give the same result.
+template <int D, bool BRANCH_FREE_MASK>
 __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint32_t o_col, float sl2, bool edge,
                                              int c_lo, int c_hi, float& m_used, float& l, bool o_live) {
 #if HSWA_SOFTMAX_SINGLE_PASS
@@ -60,9 +63,20 @@ __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint
     reg_fence_into<64>(v);
     reg_fence_into<96>(v);
     if (edge) {
+      if (BRANCH_FREE_MASK) {
+        // the sign of (k - c_lo) | (c_hi - k) is set exactly outside [c_lo, c_hi] (positions
+        // stay below 2^31 - 256, so neither difference overflows)
+        const int nlo = -c_lo;
 #pragma unroll
-      for (int k = 0; k < 128; ++k)
-        if (k < c_lo || k > c_hi) v[k] = __float_as_uint(-INFINITY);
+        for (int k = 0; k < 128; ++k) {
+          const uint32_t m = (uint32_t)(((k + nlo) | (c_hi - k)) >> 31);
+          v[k] = (v[k] & ~m) | (0xFF800000u & m);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k < c_lo || k > c_hi) v[k] = __float_as_uint(-INFINITY);
+      }
     }
     float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
     float m2 = __uint_as_float(v[2]), m3 = __uint_as_float(v[3]);
@@ -141,8 +155,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint
       if (edge) {
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          if (h2 + k < c_lo || h2 + k > c_hi) va[k] = __float_as_uint(-INFINITY);
-          if (h2 + 32 + k < c_lo || h2 + 32 + k > c_hi) vb[k] = __float_as_uint(-INFINITY);
+          const uint32_t ma = (uint32_t)(((h2 + k - c_lo) | (c_hi - h2 - k)) >> 31);
+          const uint32_t mb = (uint32_t)(((h2 + 32 + k - c_lo) | (c_hi - h2 - 32 - k)) >> 31);
+          va[k] = (va[k] & ~ma) | (0xFF800000u & ma);
+          vb[k] = (vb[k] & ~mb) | (0xFF800000u & mb);
         }
       }
       float m0 = mx, m1 = __uint_as_float(va[0]), m2 = __uint_as_float(vb[0]);
@@ -195,8 +211,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint
       const int c0 = 32 * c;
       if (edge) {
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (c0 + k < c_lo || c0 + k > c_hi) cur[k] = __float_as_uint(-INFINITY);
+        for (int k = 0; k < 32; ++k) {
+          const uint32_t m = (uint32_t)(((c0 + k - c_lo) | (c_hi - c0 - k)) >> 31);
+          cur[k] = (cur[k] & ~m) | (0xFF800000u & m);
+        }
       }
       uint32_t pk[16];
 #pragma unroll
