@@ -187,7 +187,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
   using SM = DecSmem<D, MT>;
   constexpr int ROWS = SM::ROWS;
   constexpr int CH = D / 8;              // 16-byte chunks per row
-  constexpr int ROWS_PER_PASS = 512 / (D * 2);  // rows one warp-wide 16-byte copy covers
   extern __shared__ __align__(128) uint8_t smem[];
   float* m_w = reinterpret_cast<float*>(smem + SM::MISC_OFF);   // [4][ROWS]
   float* l_w = m_w + 4 * ROWS;                                  // [4][ROWS]

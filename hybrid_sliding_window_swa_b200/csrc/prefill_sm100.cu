@@ -10,14 +10,18 @@
 // Attention and BlockSparse": blocks outside the window are skipped); only tiles
 // that the band edge crosses are masked.
 //
+// This kernel serves full layers and sliding windows W > 129; narrower windows go to
+// prefill_narrow.cu (launch_prefill dispatches). The per-row softmax step and the output
+// epilogue are shared with it (prefill_tile.cuh).
+//
 // Work unit = 2 query tiles of 128 rows (one batch row b, one query head h). The grid
 // is persistent (one CTA per SM) and walks the units in a static round-robin, heaviest
 // (latest query tiles) first; consecutive CTAs take the query heads of one KV group
 // so their K/V tiles are shared through L2.
 //   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one thread per
 //               row (TMEM lane); all 128 scores of a row in registers, online max/sum
-//               in the exp2 domain with lazy O rescaling, exponentials split between
-//               the MUFU unit and an FMA-pipe polynomial, P written back over S as
+//               in the exp2 domain with lazy O rescaling, MUFU exponentials (an FMA-pipe
+//               polynomial can take a share, HSWA_POLY_PER8), P written back over S as
 //               packed bf16, and the epilogue (O / l -> bf16, staged in shared memory per
 //               warp and written by TMA stores).
 //   warps 8-11  a third warpgroup that gives its registers to the softmax warpgroups
@@ -56,7 +60,6 @@ struct Params {
   const int32_t* seq_ids;
   const int32_t* page_table;
   int pt_stride;
-  uint16_t* o;
   const uint16_t* ring_k;
   const uint16_t* ring_v;
   int ring_layer, n_swa, max_seqs, ring_tma;
@@ -533,7 +536,6 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
   p.seq_ids = Lc.seq_ids;
   p.page_table = Lc.page_table;
   p.pt_stride = Lc.pt_stride;
-  p.o = Lc.o;
   p.ring_k = pool->ring_k;
   p.ring_v = pool->ring_v;
   p.ring_layer = Lc.ring_layer;
