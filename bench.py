@@ -732,7 +732,56 @@ def decode_results(hs, oracle_mod, hbm):
     ref = oracle_mod.window_safe_len(M.numpy(), C.numpy(), bits, W)
     res.append({"workload": "window_safe_len_4096req_W128", "metric": "latency", "unit": "us", "value": round(us, 2),
                 "requests_per_s": round(nr / (us * 1e-6)), "bit_exact": bool(np.array_equal(outw.cpu().numpy(), ref))})
+    res.append(prefix_cache_result(hs, oracle_mod))
     return res
+
+
+def prefix_cache_result(hs, oracle_mod, nr=4096, W=128, max_len=2048):
+    """SWA-aware prefix cache (host code): nr cached sequences of lengths C in [0, max_len] with
+    their own tokens, evictions following the window_safe_len request recipe, then nr matches.
+    With one sequence per path the window-safe length equals window_safe_len(m, C, mask), which
+    the oracle computes in closed form (bit-exact check over every request)."""
+    C = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 21), nr, 0, max_len).numpy()
+    M = np.where(synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 22), nr, 0, 1).numpy() == 0, C,
+                 synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 23), nr, 0, max_len).numpy())
+    ev = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 24), nr, 0, W - 1).numpy()
+    kind = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 25), nr, 0, 3).numpy()
+    bits = np.full((nr, W // 32), 0xFFFFFFFF, dtype=np.uint32)
+    tree = hs.PrefixTree(W)
+    seqs = []
+    t0 = time.perf_counter()
+    for r in range(nr):
+        seq = np.arange(int(C[r]), dtype=np.int32) + np.int32(r * 65536)  # tokens of this sequence only
+        seqs.append(seq)
+        tree.insert(seq)
+    t_insert = time.perf_counter() - t0
+    for r in range(nr):
+        s = int(C[r]) % W if kind[r] == 3 else (int(ev[r]) if kind[r] == 2 else -1)
+        if s < 0:
+            continue
+        bits[r, s // 32] &= np.uint32(~(1 << (s % 32)) & 0xFFFFFFFF)
+        for p in range(max(0, int(C[r]) - W), int(C[r])):  # the window position in that slot
+            if p % W == s:
+                tree.evict_swa(seqs[r], p, p + 1)
+    queries = []
+    for r in range(nr):
+        k = min(int(M[r]), int(C[r]))
+        extra = np.full(int(M[r]) - k, -1, dtype=np.int32)  # a token no cached sequence holds
+        queries.append(np.concatenate([seqs[r][:k], extra]))
+    times = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        m_len, safe = tree.match_batch(queries)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    ref = oracle_mod.window_safe_len(M.astype(np.int64), C.astype(np.int64), bits, W)
+    n_pos, n_held = tree.stats()
+    tree.close()
+    return {"workload": f"prefix_cache_match_{nr}req_W{W}_len{max_len}", "metric": "host match latency", "unit": "us",
+            "value": round(sec * 1e6, 1), "requests_per_s": round(nr / sec), "matched_tokens": int(m_len.sum()),
+            "ns_per_matched_token": round(sec * 1e9 / max(1, int(m_len.sum())), 1), "cached_positions": n_pos,
+            "positions_holding_swa_kv": n_held, "insert_s": round(t_insert, 3),
+            "bit_exact": bool(np.array_equal(safe, ref)), "where": "host CPU, one thread"}
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)

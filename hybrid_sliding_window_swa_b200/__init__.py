@@ -29,7 +29,8 @@ EXPORTED = [
     "kv_pool_layout", "kv_pool_create", "kv_pool_destroy", "kv_pool_append",
     "swa_prefill_fwd", "full_prefill_fwd", "hybrid_decode_workspace_size", "hybrid_decode_fwd",
     "window_safe_len", "hswa_pool_check_error", "hswa_last_error", "hybrid_decode_fwd_noalloc",
-    "hswa_selftest_wait_timeout",
+    "hswa_selftest_wait_timeout", "hswa_tree_create", "hswa_tree_destroy", "hswa_tree_insert",
+    "hswa_tree_release", "hswa_tree_evict_swa", "hswa_tree_match", "hswa_tree_match_batch", "hswa_tree_stats",
 ]
 
 # scratch bytes available to hybrid_decode_fwd_noalloc (HSWA_NOALLOC_SCRATCH_BYTES in hswa.h)
@@ -77,6 +78,14 @@ def load_library(path: str | None = None):
         "hswa_pool_check_error": [p, ctypes.POINTER(ctypes.c_int)],
         "hybrid_decode_fwd_noalloc": [p, i32, p, p, p, p, i32, i32, p, i64, p, p, i32, i32, p],
         "hswa_selftest_wait_timeout": [p, i64, p],
+        "hswa_tree_create": [ctypes.c_int32, ctypes.POINTER(p)],
+        "hswa_tree_destroy": [p],
+        "hswa_tree_insert": [p, p, i64, ctypes.POINTER(i64)],
+        "hswa_tree_release": [p, p, i64],
+        "hswa_tree_evict_swa": [p, p, i64, i64, i64, ctypes.POINTER(i64)],
+        "hswa_tree_match": [p, p, i64, ctypes.POINTER(i64), ctypes.POINTER(i64)],
+        "hswa_tree_match_batch": [p, p, p, ctypes.c_int32, p, p],
+        "hswa_tree_stats": [p, ctypes.POINTER(i64), ctypes.POINTER(i64)],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -310,3 +319,75 @@ def hybrid_decode_fwd_noalloc(pool: KVPool, layer: int, q: torch.Tensor, k_new: 
         _ptr(ctx_len, torch.int64, "ctx_len"), max_ctx_len, _ptr(seq_ids, torch.int32, "seq_ids"),
         _ptr(page_table, torch.int32, "page_table"), pt_stride, hq, _stream(stream)))
     return o
+
+
+def _tokens(tokens):
+    """int32 host token array (numpy view, or a copy when the input is not int32/contiguous)."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(tokens), dtype=np.int32)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+class PrefixTree:
+    """SWA-aware prefix cache over a token trie (host code; see include/hswa.h, hswa_tree_*)."""
+
+    def __init__(self, window: int):
+        h = ctypes.c_void_p()
+        _check(load_library().hswa_tree_create(window, ctypes.byref(h)))
+        self.handle, self.window = h, window
+
+    def close(self):
+        if self.handle:
+            load_library().hswa_tree_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def insert(self, tokens) -> int:
+        a, ptr = _tokens(tokens)
+        added = ctypes.c_int64()
+        _check(load_library().hswa_tree_insert(self.handle, ptr, a.size, ctypes.byref(added)))
+        return added.value
+
+    def release(self, tokens):
+        a, ptr = _tokens(tokens)
+        _check(load_library().hswa_tree_release(self.handle, ptr, a.size))
+
+    def evict_swa(self, tokens, pos_lo: int, pos_hi: int) -> int:
+        a, ptr = _tokens(tokens)
+        n = ctypes.c_int64()
+        _check(load_library().hswa_tree_evict_swa(self.handle, ptr, a.size, pos_lo, pos_hi, ctypes.byref(n)))
+        return n.value
+
+    def match(self, tokens) -> tuple[int, int]:
+        """(match length, window-safe length) of one request."""
+        a, ptr = _tokens(tokens)
+        m, s = ctypes.c_int64(), ctypes.c_int64()
+        _check(load_library().hswa_tree_match(self.handle, ptr, a.size, ctypes.byref(m), ctypes.byref(s)))
+        return m.value, s.value
+
+    def match_batch(self, requests):
+        """(match lengths, window-safe lengths) as int64 numpy arrays for a list of token sequences."""
+        import numpy as np
+        lens = np.array([len(r) for r in requests], dtype=np.int64)
+        offsets = np.zeros(len(requests) + 1, dtype=np.int64)
+        np.cumsum(lens, out=offsets[1:])
+        flat = np.ascontiguousarray(np.concatenate([np.asarray(r, dtype=np.int32) for r in requests])
+                                    if requests else np.zeros(0, np.int32), dtype=np.int32)
+        m = np.zeros(len(requests), dtype=np.int64)
+        s = np.zeros(len(requests), dtype=np.int64)
+        _check(load_library().hswa_tree_match_batch(
+            self.handle, flat.ctypes.data_as(ctypes.c_void_p), offsets.ctypes.data_as(ctypes.c_void_p),
+            len(requests), m.ctypes.data_as(ctypes.c_void_p), s.ctypes.data_as(ctypes.c_void_p)))
+        return m, s
+
+    def stats(self) -> tuple[int, int]:
+        """(cached positions, positions holding sliding-window KV)."""
+        n, h = ctypes.c_int64(), ctypes.c_int64()
+        _check(load_library().hswa_tree_stats(self.handle, ctypes.byref(n), ctypes.byref(h)))
+        return n.value, h.value
+

@@ -10,7 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhswa.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["hswa_abi.cu", "pool_kernels.cu", "prefill_sm100.cu", "prefill_narrow.cu", "decode.cu"]
+SOURCES = ["hswa_abi.cu", "pool_kernels.cu", "prefill_sm100.cu", "prefill_narrow.cu", "decode.cu",
+           "prefix_tree.cpp"]
 HEADERS = ["common.cuh", "internal.h", "prefill_tile.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -41,7 +42,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     jobs = []
     for src in SOURCES:
         sp = os.path.join(CSRC, src)
-        op = os.path.join(BUILD_DIR, src.replace(".cu", ".o"))
+        op = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
         objs.append(op)
         if force or _stale(op, [sp] + hdrs):
             cmd = [NVCC, *FLAGS, *[f"-D{d}" for d in defines], "-c", sp, "-o", op]

@@ -204,6 +204,48 @@ HSWA_API int window_safe_len(const int64_t* match_len, const int64_t* cached_len
                     const uint32_t* slot_valid, int32_t W, int32_t n_req, int64_t* out_len,
                     void* stream);
 
+/* SWA-aware prefix cache over a token trie (host memory, host code; "MiMo v2.5 inference
+ * optimisation", section "KV cache redesign": a prefix-cache match is cut to the window-safe
+ * length, since with sliding-window layers only part of a cached sequence's window KV may
+ * survive). Each trie node is one cached position. Its full-attention KV is held while the node
+ * exists; its sliding-window KV is held while at least one cached sequence's window (its last W
+ * positions) covers it and it has not been evicted. With one cached sequence this is
+ * window_safe_len with a per-position eviction mask; here cached sequences share prefixes.
+ * Token ids are any int32 values. Calls on one tree are not thread-safe; the caller serialises
+ * them. Errors: HSWA_ERR_INVALID_ARG for null pointers or negative lengths,
+ * HSWA_ERR_OUT_OF_MEMORY when the host allocation fails (the tree is left valid). */
+typedef struct hswa_prefix_tree hswa_prefix_tree;
+
+/* New empty tree for window W >= 1; *out owns host memory until hswa_tree_destroy. */
+HSWA_API int hswa_tree_create(int32_t window, hswa_prefix_tree** out);
+HSWA_API int hswa_tree_destroy(hswa_prefix_tree* tree);
+
+/* Cache tokens[0..n): adds the missing positions and counts this sequence's window
+ * [max(0, n-W), n) as holding sliding-window KV. *new_nodes (may be null) = positions added. */
+HSWA_API int hswa_tree_insert(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int64_t* new_nodes);
+
+/* Undo one hswa_tree_insert of the same tokens: its window stops counting (positions shared
+ * with other cached windows stay held). HSWA_ERR_INVALID_ARG if the sequence is not in the tree. */
+HSWA_API int hswa_tree_release(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n);
+
+/* Drop the sliding-window KV of positions [pos_lo, pos_hi) along the path tokens[0..n) (all
+ * cached windows that cover them lose it); *evicted (may be null) = positions that held it. */
+HSWA_API int hswa_tree_evict_swa(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int64_t pos_lo,
+                                 int64_t pos_hi, int64_t* evicted);
+
+/* Match tokens[0..n): *match_len = m = longest cached prefix; *safe_len = max { L in [0, m] :
+ * every position in [max(0, L-W), L) holds sliding-window KV }, the length a request can resume
+ * from. Exact integers. */
+HSWA_API int hswa_tree_match(const hswa_prefix_tree* tree, const int32_t* tokens, int64_t n,
+                             int64_t* match_len, int64_t* safe_len);
+
+/* hswa_tree_match for n_req requests: request r is tokens[offsets[r] .. offsets[r+1]). */
+HSWA_API int hswa_tree_match_batch(const hswa_prefix_tree* tree, const int32_t* tokens, const int64_t* offsets,
+                                   int32_t n_req, int64_t* match_len, int64_t* safe_len);
+
+/* Cached positions (trie nodes) and how many of them hold sliding-window KV. */
+HSWA_API int hswa_tree_stats(const hswa_prefix_tree* tree, int64_t* n_positions, int64_t* n_swa_held);
+
 /* Diagnostic: run, on `stream`, one wait on a barrier that nothing arrives at, through the same
  * bounded wait every kernel uses, with a limit of limit_ns (1 ms .. 2 s; the kernels themselves
  * use 2 s). The wait gives up, records HSWA_ERR_TIMEOUT in the pool's error word and the kernel

@@ -4,7 +4,8 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` and
 ``--impl reference`` legs of ``bench.py`` may import this package. The product
 path (``hybrid_sliding_window_swa_b200``) never imports it and shares no code
 with it. The arithmetic lives in ``oracle.c`` (plain C, fp64); this module only
-builds it with gcc and marshals numpy/torch arrays through ctypes.
+builds it with gcc and marshals numpy/torch arrays through ctypes, except for
+``prefix_cache_replay``, a brute-force integer model written out in Python.
 
 Every function here restates a passage of the source pages; see ``oracle.h``
 for the citations and the readings taken where the pages are silent.
@@ -140,3 +141,53 @@ def pool_bytes(n_swa_layers: int, n_full_layers: int, window: int, n_kv_heads: i
     swa = kv_bytes(n_swa_layers, n_kv_heads, window * max_seqs, head_dim, elem_bytes)
     full = kv_bytes(n_full_layers, n_kv_heads, pages_per_full_layer * page_size, head_dim, elem_bytes)
     return swa, full
+
+
+def prefix_cache_replay(window: int, ops):
+    """Brute-force model of the SWA-aware prefix cache ("MiMo v2.5 inference optimisation",
+    section "KV cache redesign": a prefix-cache match is cut to the window-safe length because
+    only part of a cached sequence's window KV may survive).
+
+    State, by definition: a cached position is a token prefix (a tuple); every cached position
+    keeps its full-attention KV; its sliding-window KV is held while the number of cached
+    sequences whose last `window` positions include it is positive and it was not evicted since.
+    `ops` is a list of ("insert", tokens), ("release", tokens), ("evict", tokens, lo, hi) and
+    ("match", tokens); returns, for each "match" in order, (m, L): m = the longest cached prefix
+    of tokens, L = max { L in [0, m] : every position in [max(0, L - window), L) holds its
+    sliding-window KV }. Quadratic in sequence length: for small cases only.
+    """
+    cached = set()
+    refs = {}
+    out = []
+    for op in ops:
+        kind, toks = op[0], tuple(int(t) for t in op[1])
+        n = len(toks)
+        win = range(max(0, n - window), n)
+        if kind == "insert":
+            for p in range(n):
+                cached.add(toks[:p + 1])
+            for p in win:
+                refs[toks[:p + 1]] = refs.get(toks[:p + 1], 0) + 1
+        elif kind == "release":
+            assert toks[:n] in cached or n == 0, "release of a sequence that is not cached"
+            for p in win:
+                key = toks[:p + 1]
+                refs[key] = max(0, refs.get(key, 0) - 1)
+        elif kind == "evict":
+            lo, hi = op[2], op[3]
+            for p in range(max(0, lo), min(n, hi)):
+                if toks[:p + 1] in cached:
+                    refs[toks[:p + 1]] = 0
+        elif kind == "match":
+            m = 0
+            while m < n and toks[:m + 1] in cached:
+                m += 1
+            best = 0
+            for L in range(0, m + 1):
+                if all(refs.get(toks[:q + 1], 0) > 0 for q in range(max(0, L - window), L)):
+                    best = L
+            out.append((m, best))
+        else:
+            raise ValueError(kind)
+    return out
+
