@@ -12,6 +12,7 @@
 //
 // With one cached sequence of length C this reduces to window_safe_len (a ring of W slots holding
 // positions [max(0, C - W), C)); here eviction is per position and cached sequences share prefixes.
+#include <algorithm>
 #include <cstdint>
 #include <new>
 #include <unordered_map>
@@ -24,18 +25,54 @@ void set_error(const char* fmt, ...);
 }
 
 struct hswa_prefix_tree {
+  // Path-compressed trie: node k holds a run of consecutive cached positions (its label) and,
+  // per position, the number of cached windows holding sliding-window KV there (0 after an
+  // eviction). Node 0 is the root with an empty label. A child is found by (node, first token).
+  struct Node {
+    int64_t pos0;                 // position of the label's first token
+    std::vector<int32_t> label;   // tokens at positions pos0 .. pos0 + label.size() - 1
+    std::vector<uint32_t> refs;   // per position of the label
+    std::vector<int32_t> kids;    // children (their first tokens key the lookup map)
+  };
   int32_t window;
-  // node 0 is the root (no token); node k > 0 is one position: depth[k] = position + 1
-  std::vector<int32_t> parent;
-  std::vector<int32_t> token;
-  std::vector<int64_t> depth;
-  std::vector<uint32_t> swa_refs;  // cached sequences whose window covers this position (0 after eviction)
-  std::unordered_map<uint64_t, int32_t> child;  // (parent, token) -> node
+  std::vector<Node> nodes;
+  std::unordered_map<uint64_t, int32_t> child;  // (node, first token of the child's label) -> child
+  int64_t n_positions = 0;
 
-  static uint64_t key(int32_t p, int32_t t) { return ((uint64_t)(uint32_t)p << 32) | (uint32_t)t; }
-  int32_t find(int32_t p, int32_t t) const {
-    auto it = child.find(key(p, t));
+  static uint64_t key(int32_t n, int32_t t) { return ((uint64_t)(uint32_t)n << 32) | (uint32_t)t; }
+  int32_t find(int32_t n, int32_t t) const {
+    auto it = child.find(key(n, t));
     return it == child.end() ? -1 : it->second;
+  }
+
+  // Visit the cached positions along tokens[0..n) in order, as runs inside node labels:
+  // f(node, offset in label, position, run length). Stops where the path leaves the tree;
+  // returns the number of positions visited (the common-prefix length).
+  template <class F>
+  int64_t walk(const int32_t* tokens, int64_t n, F&& f) {
+    int32_t node = 0;
+    size_t off = 0;  // offset inside the current node's label; the root's label is empty
+    int64_t i = 0;
+    while (i < n) {
+      Node* nd = &nodes[node];
+      if (off == nd->label.size()) {
+        const int32_t c = find(node, tokens[i]);
+        if (c < 0) break;
+        node = c;
+        off = 0;
+        nd = &nodes[node];
+      }
+      // longest run of equal tokens inside this label
+      const size_t lim = std::min<size_t>(nd->label.size() - off, (size_t)(n - i));
+      size_t k = 0;
+      while (k < lim && nd->label[off + k] == tokens[i + k]) ++k;
+      if (k == 0) break;
+      f(node, off, i, (int64_t)k);
+      off += k;
+      i += (int64_t)k;
+      if (off < nd->label.size()) break;  // diverged (or ran out of tokens) inside the label
+    }
+    return i;
   }
 };
 
@@ -64,10 +101,7 @@ int hswa_tree_create(int32_t window, hswa_prefix_tree** out) {
     return HSWA_ERR_OUT_OF_MEMORY;
   }
   t->window = window;
-  t->parent.push_back(-1);
-  t->token.push_back(0);
-  t->depth.push_back(0);
-  t->swa_refs.push_back(0);
+  t->nodes.push_back(hswa_prefix_tree::Node{0, {}, {}, {}});
   *out = t;
   return HSWA_OK;
 }
@@ -83,32 +117,78 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
     return HSWA_ERR_INVALID_ARG;
   }
   if (!check_tokens(tokens, n, "hswa_tree_insert")) return HSWA_ERR_INVALID_ARG;
-  if ((int64_t)t->parent.size() + n > INT32_MAX) {
-    hswa::set_error("hswa_tree_insert: tree would exceed 2^31 nodes");
-    return HSWA_ERR_OUT_OF_MEMORY;
-  }
   int64_t added = 0;
-  int32_t node = 0;
-  const int64_t win_lo = n > t->window ? n - t->window : 0;
   try {
-    for (int64_t p = 0; p < n; ++p) {
-      int32_t c = t->find(node, tokens[p]);
-      if (c < 0) {
-        c = (int32_t)t->parent.size();
-        t->parent.push_back(node);
-        t->token.push_back(tokens[p]);
-        t->depth.push_back(p + 1);
-        t->swa_refs.push_back(0);
-        t->child.emplace(hswa_prefix_tree::key(node, tokens[p]), c);
-        ++added;
+    // 1. structure: follow the cached prefix, split the label where the path leaves it, and
+    //    attach the rest of the sequence as one new node
+    int32_t node = 0;
+    size_t off = 0;
+    int64_t i = 0;
+    while (i < n) {
+      hswa_prefix_tree::Node* nd = &t->nodes[node];
+      if (off == nd->label.size()) {
+        const int32_t c = t->find(node, tokens[i]);
+        if (c < 0) break;
+        node = c;
+        off = 0;
+        continue;
       }
-      if (p >= win_lo) ++t->swa_refs[c];  // this sequence's window: its last W positions
-      node = c;
+      if (nd->label[off] != tokens[i]) {
+        // split node at off: the head keeps [0, off), a new tail node takes the rest and the
+        // old children
+        if (t->nodes.size() >= (size_t)INT32_MAX - 2) {
+          hswa::set_error("hswa_tree_insert: tree would exceed 2^31 nodes");
+          return HSWA_ERR_OUT_OF_MEMORY;
+        }
+        const int32_t tail = (int32_t)t->nodes.size();
+        hswa_prefix_tree::Node tn;
+        tn.pos0 = nd->pos0 + (int64_t)off;
+        tn.label.assign(nd->label.begin() + off, nd->label.end());
+        tn.refs.assign(nd->refs.begin() + off, nd->refs.end());
+        t->nodes.push_back(std::move(tn));
+        nd = &t->nodes[node];  // the vector may have moved
+        // the old children now hang under the tail node
+        t->nodes[tail].kids.swap(nd->kids);
+        for (int32_t c : t->nodes[tail].kids) {
+          const int32_t tok = t->nodes[c].label[0];
+          t->child.erase(hswa_prefix_tree::key(node, tok));
+          t->child[hswa_prefix_tree::key(tail, tok)] = c;
+        }
+        nd->kids.assign(1, tail);
+        t->child[hswa_prefix_tree::key(node, t->nodes[tail].label[0])] = tail;
+        nd->label.resize(off);
+        nd->refs.resize(off);
+        break;
+      }
+      ++off;
+      ++i;
+    }
+    if (i < n) {
+      if (t->nodes.size() >= (size_t)INT32_MAX - 2) {
+        hswa::set_error("hswa_tree_insert: tree would exceed 2^31 nodes");
+        return HSWA_ERR_OUT_OF_MEMORY;
+      }
+      const int32_t fresh = (int32_t)t->nodes.size();
+      hswa_prefix_tree::Node fn;
+      fn.pos0 = i;
+      fn.label.assign(tokens + i, tokens + n);
+      fn.refs.assign((size_t)(n - i), 0u);
+      t->nodes.push_back(std::move(fn));
+      t->nodes[node].kids.push_back(fresh);
+      t->child[hswa_prefix_tree::key(node, tokens[i])] = fresh;
+      added = n - i;
+      t->n_positions += added;
     }
   } catch (const std::bad_alloc&) {
     hswa::set_error("hswa_tree_insert: out of host memory");
     return HSWA_ERR_OUT_OF_MEMORY;
   }
+  // 2. this sequence's window, its last W positions, now holds sliding-window KV
+  const int64_t win_lo = n > t->window ? n - t->window : 0;
+  t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    for (int64_t k = 0; k < len; ++k)
+      if (pos + k >= win_lo) ++t->nodes[node].refs[off + (size_t)k];
+  });
   if (new_nodes) *new_nodes = added;
   return HSWA_OK;
 }
@@ -119,16 +199,17 @@ int hswa_tree_release(hswa_prefix_tree* t, const int32_t* tokens, int64_t n) {
     return HSWA_ERR_INVALID_ARG;
   }
   if (!check_tokens(tokens, n, "hswa_tree_release")) return HSWA_ERR_INVALID_ARG;
-  const int64_t win_lo = n > t->window ? n - t->window : 0;
-  int32_t node = 0;
-  for (int64_t p = 0; p < n; ++p) {
-    node = t->find(node, tokens[p]);
-    if (node < 0) {
-      hswa::set_error("hswa_tree_release: sequence is not cached");
-      return HSWA_ERR_INVALID_ARG;
-    }
-    if (p >= win_lo && t->swa_refs[node] > 0) --t->swa_refs[node];
+  if (t->walk(tokens, n, [](int32_t, size_t, int64_t, int64_t) {}) != n) {
+    hswa::set_error("hswa_tree_release: sequence is not cached");
+    return HSWA_ERR_INVALID_ARG;
   }
+  const int64_t win_lo = n > t->window ? n - t->window : 0;
+  t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    for (int64_t k = 0; k < len; ++k) {
+      uint32_t& r = t->nodes[node].refs[off + (size_t)k];
+      if (pos + k >= win_lo && r > 0) --r;
+    }
+  });
   return HSWA_OK;
 }
 
@@ -140,38 +221,37 @@ int hswa_tree_evict_swa(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, i
   }
   if (!check_tokens(tokens, n, "hswa_tree_evict_swa")) return HSWA_ERR_INVALID_ARG;
   int64_t count = 0;
-  int32_t node = 0;
-  for (int64_t p = 0; p < n && p < pos_hi; ++p) {
-    node = t->find(node, tokens[p]);
-    if (node < 0) break;  // positions past the cached part hold nothing to evict
-    if (p >= pos_lo && t->swa_refs[node] > 0) {
-      t->swa_refs[node] = 0;
-      ++count;
+  t->walk(tokens, n < pos_hi ? n : (pos_hi > 0 ? pos_hi : 0), [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    for (int64_t k = 0; k < len; ++k) {
+      uint32_t& r = t->nodes[node].refs[off + (size_t)k];
+      if (pos + k >= pos_lo && r > 0) {
+        r = 0;
+        ++count;
+      }
     }
-  }
+  });
   if (evicted) *evicted = count;
   return HSWA_OK;
 }
 
-int hswa_tree_match(const hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int64_t* match_len,
+int hswa_tree_match(const hswa_prefix_tree* tc, const int32_t* tokens, int64_t n, int64_t* match_len,
                     int64_t* safe_len) {
-  if (!t || !match_len || !safe_len) {
+  if (!tc || !match_len || !safe_len) {
     hswa::set_error("hswa_tree_match: null argument");
     return HSWA_ERR_INVALID_ARG;
   }
   if (!check_tokens(tokens, n, "hswa_tree_match")) return HSWA_ERR_INVALID_ARG;
-  // walk the common prefix; run = consecutive held positions ending at p
+  hswa_prefix_tree* t = const_cast<hswa_prefix_tree*>(tc);  // walk() only reads
   const int64_t W = t->window;
-  int32_t node = 0;
-  int64_t m = 0, run = 0, best = 0;
-  for (int64_t p = 0; p < n; ++p) {
-    node = t->find(node, tokens[p]);
-    if (node < 0) break;
-    m = p + 1;
-    run = t->swa_refs[node] > 0 ? run + 1 : 0;
-    // L = p + 1 is safe when its tail [max(0, L - W), L) is held
-    if (run >= (m < W ? m : W)) best = m;
-  }
+  int64_t run = 0, best = 0;  // run: consecutive positions holding sliding-window KV
+  const int64_t m = t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    const uint32_t* r = t->nodes[node].refs.data() + off;
+    for (int64_t k = 0; k < len; ++k) {
+      run = r[k] > 0 ? run + 1 : 0;
+      const int64_t L = pos + k + 1;  // safe when its tail [max(0, L - W), L) is held
+      if (run >= (L < W ? L : W)) best = L;
+    }
+  });
   *match_len = m;
   *safe_len = best;
   return HSWA_OK;
@@ -201,8 +281,9 @@ int hswa_tree_stats(const hswa_prefix_tree* t, int64_t* n_positions, int64_t* n_
     return HSWA_ERR_INVALID_ARG;
   }
   int64_t held = 0;
-  for (size_t k = 1; k < t->swa_refs.size(); ++k) held += t->swa_refs[k] > 0;
-  if (n_positions) *n_positions = (int64_t)t->parent.size() - 1;
+  for (const auto& nd : t->nodes)
+    for (uint32_t r : nd.refs) held += r > 0;
+  if (n_positions) *n_positions = t->n_positions;
   if (n_swa_held) *n_swa_held = held;
   return HSWA_OK;
 }
