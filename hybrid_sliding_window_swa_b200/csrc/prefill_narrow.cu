@@ -299,6 +299,8 @@ __device__ void softmax_slot(const NParams& p, uint8_t* smem, NBars* bars, uint3
     NGeo G;
     make_ngeo(p, unit, G);
     const int lo_last = nwindow_lo(p, G.i1);
+    // W = 128 and no row's band clipped at the sequence start: the rotated-chunk mask applies
+    const bool w128 = p.window == 128 && G.nkt == 2 && G.i0 >= 127 && G.jlo == G.t - 1;
     const int i = G.i0 + r;
     const int lo_i = nwindow_lo(p, i);
     for (int k = 0; k < G.nh[q]; ++k) {
@@ -311,7 +313,10 @@ __device__ void softmax_slot(const NParams& p, uint8_t* smem, NBars* bars, uint3
         // columns of this row inside the band: [c_lo, c_hi] (edge tiles only)
         const int kb = G.P + BN * (G.jlo + jj);
         const bool edge = !(kb + BN - 1 <= G.i0 && kb >= lo_last);
-        softmax_tile<D, false>(trow, s_col, o_col, sl2, edge, lo_i - kb, i - kb, m_used, l, jj > 0);
+        if (w128)
+          softmax_tile<D, 2>(trow, s_col, o_col, sl2, true, 0, 0, m_used, l, jj > 0, wq, jj == 0);
+        else
+          softmax_tile<D, 0>(trow, s_col, o_col, sl2, edge, lo_i - kb, i - kb, m_used, l, jj > 0);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_full[q]);

@@ -429,7 +429,7 @@ __device__ void softmax_wg(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
       const bool edge = !(kb + BN - 1 <= qi0 && kb >= lo_last);
       const int c_lo = lo_i - kb;
       const int c_hi = i - kb;
-      softmax_tile<D, true>(trow, s_col, o_col, sl2, edge, c_lo, c_hi, m_used, l, n_done > 0);
+      softmax_tile<D, 1>(trow, s_col, o_col, sl2, edge, c_lo, c_hi, m_used, l, n_done > 0);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[q]);

@@ -44,25 +44,55 @@ __device__ __forceinline__ constexpr bool use_poly(int pair) { return (pair & 7)
 // `edge`. m_used / l: running maximum (log2 domain) and row sum; o_live: O already holds a
 // partial sum (it is rescaled when the maximum moves). P is written over S as packed bf16;
 // the caller waits for the TMEM stores and signals the MMA.
-// BRANCH_FREE_MASK selects how edge tiles are masked: integer sign arithmetic on every column
-// (faster where edge tiles are few, as in long windows) or per-column compares (faster where
-// every tile is an edge tile, as in the narrow-window kernel); both give the same result.
-template <int D, bool BRANCH_FREE_MASK>
+// MASK_MODE selects how edge tiles are masked (all give the same result):
+//  0  per-column compares (faster where every tile is an edge tile, as in the narrow kernel);
+//  1  integer sign arithmetic on every column (faster where edge tiles are few);
+//  2  W = 128 with no row's band clipped at the sequence start (the narrow kernel's common tile):
+//     before the diagonal a row keeps columns k > r, on the diagonal k <= r, so for warp w
+//     (rows 32w .. 32w + 31) chunk w is the only chunk the band edge crosses and every other
+//     chunk is wholly in or out for the whole warp. The warp loads chunk (w + c) & 3 into
+//     register block c (rot = w), masks block 0 by lane and selects the other blocks whole;
+//     `lower_edge` marks the tile before the diagonal. Single-pass softmax only.
+template <int D, int MASK_MODE>
 __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint32_t o_col, float sl2, bool edge,
-                                             int c_lo, int c_hi, float& m_used, float& l, bool o_live) {
+                                             int c_lo, int c_hi, float& m_used, float& l, bool o_live,
+                                             int rot = 0, bool lower_edge = false) {
+  static_assert(MASK_MODE != 2 || HSWA_SOFTMAX_SINGLE_PASS, "the rotated mask needs the single-pass softmax");
+  constexpr bool BRANCH_FREE_MASK = MASK_MODE == 1;
+  const int rc = MASK_MODE == 2 ? rot : 0;  // chunk rotation (0 folds away in the other modes)
 #if HSWA_SOFTMAX_SINGLE_PASS
     // all 128 scores of the row: four TMEM loads, one wait
     uint32_t v[128];
-    tmem_ld32_into<0>(trow + s_col + 0, v);
-    tmem_ld32_into<32>(trow + s_col + 32, v);
-    tmem_ld32_into<64>(trow + s_col + 64, v);
-    tmem_ld32_into<96>(trow + s_col + 96, v);
+    tmem_ld32_into<0>(trow + s_col + 32 * ((rc + 0) & 3), v);
+    tmem_ld32_into<32>(trow + s_col + 32 * ((rc + 1) & 3), v);
+    tmem_ld32_into<64>(trow + s_col + 32 * ((rc + 2) & 3), v);
+    tmem_ld32_into<96>(trow + s_col + 32 * ((rc + 3) & 3), v);
     tmem_wait_ld();
     reg_fence_into<0>(v);
     reg_fence_into<32>(v);
     reg_fence_into<64>(v);
     reg_fence_into<96>(v);
-    if (edge) {
+    if (MASK_MODE == 2) {
+      // block 0 = chunk rot: the lower edge keeps j > lane, the diagonal keeps j <= lane
+      const int lane = threadIdx.x & 31;
+      if (lower_edge) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j <= lane) v[j] = 0xFF800000u;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j > lane) v[j] = 0xFF800000u;
+      }
+#pragma unroll
+      for (int c = 1; c < 4; ++c) {
+        // chunk rot + c lies above the warp's rows (kept before the diagonal, dropped on it);
+        // a wrapped chunk lies below them
+        const bool out = lower_edge ? (rc + c > 3) : (rc + c <= 3);
+#pragma unroll
+        for (int j = 32 * c; j < 32 * c + 32; ++j) v[j] = out ? 0xFF800000u : v[j];
+      }
+    } else if (edge) {
       if (BRANCH_FREE_MASK) {
         // the sign of (k - c_lo) | (c_hi - k) is set exactly outside [c_lo, c_hi] (positions
         // stay below 2^31 - 256, so neither difference overflows)
@@ -139,7 +169,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint
         f2_unpack(e, e0, e1);
         pk[k >> 1] = pack_bf16x2(e0, e1);
       }
-      tmem_st16(trow + s_col + (c0 >> 1), pk);
+      tmem_st16(trow + s_col + 16 * (((c0 >> 5) + rc) & 3), pk);
     }
 #else
     // pass 1: row maximum, 64 scores at a time
