@@ -152,6 +152,16 @@ __device__ __forceinline__ void softmax_tile(uint32_t trow, uint32_t s_col, uint
 #pragma unroll
     for (int c0 = 0; c0 < BN; c0 += 32) {
       uint32_t pk[16];
+      if (MASK_MODE == 2 && c0 > 0) {
+        // a block wholly outside every row's band: P = 0 without exponentials
+        const bool out = lower_edge ? (rc + (c0 >> 5) > 3) : (rc + (c0 >> 5) <= 3);
+        if (out) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+          tmem_st16(trow + s_col + 16 * (((c0 >> 5) + rc) & 3), pk);
+          continue;
+        }
+      }
 #pragma unroll
       for (int k = 0; k < 32; k += 2) {
         const int pair = (c0 + k) >> 1;
