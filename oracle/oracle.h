@@ -21,8 +21,7 @@
  *    match must have valid SWA slots); section "architecture": 60 SWA + 10 full
  *    layers, KV ratio (60 W + 10 N) / (70 N).
  *
- * Readings taken where the pages are silent or garbled (each one is listed in
- * the design doc too):
+ * Readings taken where the pages are silent or garbled:
  *  - positions are 0-based (eq.(1) uses max(0, .)); eq.(4)'s k = 1..n is read as
  *    the same 0-based row;
  *  - GQA maps query head h to KV head floor(h / (Hq / Hkv));

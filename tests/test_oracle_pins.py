@@ -221,7 +221,9 @@ def test_softmax_weights_shift_invariance():
 # ---------------------------------------------------------------- window_safe_len
 
 def _closed_form_wsl(m, c, bits, w):
-    """Closed form derived from the definition (window-safe length)."""
+    """Closed form derived from the definition: with the ring holding [max(0, c - w), c), a cached
+    length above w is resumable only in full (every slot valid and m >= c), otherwise the answer is
+    min(m, c, first invalid slot)."""
     if c > w:
         return c if (m >= c and all(bits)) else 0
     first_bad = next((s for s in range(w) if not bits[s]), w)
