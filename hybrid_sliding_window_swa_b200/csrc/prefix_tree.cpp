@@ -49,12 +49,12 @@ struct hswa_prefix_tree {
   // f(node, offset in label, position, run length). Stops where the path leaves the tree;
   // returns the number of positions visited (the common-prefix length).
   template <class F>
-  int64_t walk(const int32_t* tokens, int64_t n, F&& f) {
+  int64_t walk(const int32_t* tokens, int64_t n, F&& f) const {
     int32_t node = 0;
     size_t off = 0;  // offset inside the current node's label; the root's label is empty
     int64_t i = 0;
     while (i < n) {
-      Node* nd = &nodes[node];
+      const Node* nd = &nodes[node];
       if (off == nd->label.size()) {
         const int32_t c = find(node, tokens[i]);
         if (c < 0) break;
@@ -234,14 +234,13 @@ int hswa_tree_evict_swa(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, i
   return HSWA_OK;
 }
 
-int hswa_tree_match(const hswa_prefix_tree* tc, const int32_t* tokens, int64_t n, int64_t* match_len,
+int hswa_tree_match(const hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int64_t* match_len,
                     int64_t* safe_len) {
-  if (!tc || !match_len || !safe_len) {
+  if (!t || !match_len || !safe_len) {
     hswa::set_error("hswa_tree_match: null argument");
     return HSWA_ERR_INVALID_ARG;
   }
   if (!check_tokens(tokens, n, "hswa_tree_match")) return HSWA_ERR_INVALID_ARG;
-  hswa_prefix_tree* t = const_cast<hswa_prefix_tree*>(tc);  // walk() only reads
   const int64_t W = t->window;
   int64_t run = 0, best = 0;  // run: consecutive positions holding sliding-window KV
   const int64_t m = t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {

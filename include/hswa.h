@@ -212,8 +212,9 @@ HSWA_API int window_safe_len(const int64_t* match_len, const int64_t* cached_len
  * positions) covers it and it has not been evicted. With one cached sequence this is
  * window_safe_len with a per-position eviction mask; here cached sequences share prefixes.
  * Token ids are any int32 values. Calls on one tree are not thread-safe; the caller serialises
- * them. Errors: HSWA_ERR_INVALID_ARG for null pointers or negative lengths,
- * HSWA_ERR_OUT_OF_MEMORY when the host allocation fails (the tree is left valid). */
+ * them. Errors: HSWA_ERR_INVALID_ARG for null pointers or negative lengths (nothing changes);
+ * HSWA_ERR_OUT_OF_MEMORY when a host allocation fails during an insert, after which the tree
+ * may hold part of that insert and should be destroyed. */
 typedef struct hswa_prefix_tree hswa_prefix_tree;
 
 /* New empty tree for window W >= 1; *out owns host memory until hswa_tree_destroy. */
