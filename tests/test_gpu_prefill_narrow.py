@@ -20,6 +20,8 @@ pytestmark = pytest.mark.gpu
     (384, 129, 10, 2, 128, [256, 640]),  # W = 129 (largest narrow window), prefix rows by cp.async
     (130, 2, 8, 1, 64, [5, 0]),          # W = 2, G = 8, a 2-row tail tile
     (1000, 128, 8, 1, 128, [0, 131072]), # many units, prefix far into the sequence
+    (300, 128, 8, 2, 128, [126, 127]),   # W = 128 at the rotated-mask boundary (first row 126 / 127)
+    (300, 128, 4, 1, 64, [128, 255]),    # rotated mask with an aligned and an unaligned ring prefix
 ])
 def test_narrow_window_cases(n_q, W, hq, hkv, d, starts):
     got, ref = run_swa_case(107, 2, n_q, W, hq, hkv, d, starts)
