@@ -32,6 +32,7 @@ struct hswa_prefix_tree {
     int64_t pos0;                 // position of the label's first token
     std::vector<int32_t> label;   // tokens at positions pos0 .. pos0 + label.size() - 1
     std::vector<uint32_t> refs;   // per position of the label
+    std::vector<uint32_t> ends;   // per position: inserts (not yet released) that end there
     std::vector<int32_t> kids;    // children (their first tokens key the lookup map)
   };
   int32_t window;
@@ -101,7 +102,7 @@ int hswa_tree_create(int32_t window, hswa_prefix_tree** out) {
     return HSWA_ERR_OUT_OF_MEMORY;
   }
   t->window = window;
-  t->nodes.push_back(hswa_prefix_tree::Node{0, {}, {}, {}});
+  t->nodes.push_back(hswa_prefix_tree::Node{0, {}, {}, {}, {}});
   *out = t;
   return HSWA_OK;
 }
@@ -145,6 +146,7 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
         tn.pos0 = nd->pos0 + (int64_t)off;
         tn.label.assign(nd->label.begin() + off, nd->label.end());
         tn.refs.assign(nd->refs.begin() + off, nd->refs.end());
+        tn.ends.assign(nd->ends.begin() + off, nd->ends.end());
         t->nodes.push_back(std::move(tn));
         nd = &t->nodes[node];  // the vector may have moved
         // the old children now hang under the tail node
@@ -158,6 +160,7 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
         t->child[hswa_prefix_tree::key(node, t->nodes[tail].label[0])] = tail;
         nd->label.resize(off);
         nd->refs.resize(off);
+        nd->ends.resize(off);
         break;
       }
       ++off;
@@ -173,6 +176,7 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
       fn.pos0 = i;
       fn.label.assign(tokens + i, tokens + n);
       fn.refs.assign((size_t)(n - i), 0u);
+      fn.ends.assign((size_t)(n - i), 0u);
       t->nodes.push_back(std::move(fn));
       t->nodes[node].kids.push_back(fresh);
       t->child[hswa_prefix_tree::key(node, tokens[i])] = fresh;
@@ -183,11 +187,14 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
     hswa::set_error("hswa_tree_insert: out of host memory");
     return HSWA_ERR_OUT_OF_MEMORY;
   }
-  // 2. this sequence's window, its last W positions, now holds sliding-window KV
+  // 2. this sequence's window, its last W positions, now holds sliding-window KV, and one more
+  //    insert ends at its last position
   const int64_t win_lo = n > t->window ? n - t->window : 0;
   t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
-    for (int64_t k = 0; k < len; ++k)
+    for (int64_t k = 0; k < len; ++k) {
       if (pos + k >= win_lo) ++t->nodes[node].refs[off + (size_t)k];
+      if (pos + k == n - 1) ++t->nodes[node].ends[off + (size_t)k];
+    }
   });
   if (new_nodes) *new_nodes = added;
   return HSWA_OK;
@@ -199,10 +206,17 @@ int hswa_tree_release(hswa_prefix_tree* t, const int32_t* tokens, int64_t n) {
     return HSWA_ERR_INVALID_ARG;
   }
   if (!check_tokens(tokens, n, "hswa_tree_release")) return HSWA_ERR_INVALID_ARG;
-  if (t->walk(tokens, n, [](int32_t, size_t, int64_t, int64_t) {}) != n) {
-    hswa::set_error("hswa_tree_release: sequence is not cached");
+  if (n == 0) return HSWA_OK;  // the empty sequence holds nothing
+  // the sequence must be cached and at least one insert of exactly these tokens not yet released
+  uint32_t* end_count = nullptr;
+  const int64_t m = t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    if (pos + len == n) end_count = &t->nodes[node].ends[off + (size_t)(len - 1)];
+  });
+  if (m != n || !end_count || *end_count == 0) {
+    hswa::set_error("hswa_tree_release: no insert of exactly this sequence is left to release");
     return HSWA_ERR_INVALID_ARG;
   }
+  --*end_count;
   const int64_t win_lo = n > t->window ? n - t->window : 0;
   t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
     for (int64_t k = 0; k < len; ++k) {

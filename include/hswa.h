@@ -226,7 +226,9 @@ HSWA_API int hswa_tree_destroy(hswa_prefix_tree* tree);
 HSWA_API int hswa_tree_insert(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int64_t* new_nodes);
 
 /* Undo one hswa_tree_insert of the same tokens: its window stops counting (positions shared
- * with other cached windows stay held). HSWA_ERR_INVALID_ARG if the sequence is not in the tree. */
+ * with other cached windows stay held). HSWA_ERR_INVALID_ARG, with nothing changed, unless an
+ * insert of exactly these tokens is left to undo (a cached prefix that was never inserted on its
+ * own, or a second release of a single insert, is rejected). n = 0 is a no-op. */
 HSWA_API int hswa_tree_release(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n);
 
 /* Drop the sliding-window KV of positions [pos_lo, pos_hi) along the path tokens[0..n) (all

@@ -152,12 +152,14 @@ def prefix_cache_replay(window: int, ops):
     keeps its full-attention KV; its sliding-window KV is held while the number of cached
     sequences whose last `window` positions include it is positive and it was not evicted since.
     `ops` is a list of ("insert", tokens), ("release", tokens), ("evict", tokens, lo, hi) and
-    ("match", tokens); returns, for each "match" in order, (m, L): m = the longest cached prefix
-    of tokens, L = max { L in [0, m] : every position in [max(0, L - window), L) holds its
+    ("match", tokens); a release undoes one earlier insert of exactly the same tokens (ValueError
+    when none is left; the empty sequence is a no-op); returns, for each "match" in order,
+    (m, L): m = the longest cached prefix of tokens, L = max { L in [0, m] : every position in [max(0, L - window), L) holds its
     sliding-window KV }. Quadratic in sequence length: for small cases only.
     """
     cached = set()
     refs = {}
+    inserted = {}  # exact token tuple -> inserts not yet released
     out = []
     for op in ops:
         kind, toks = op[0], tuple(int(t) for t in op[1])
@@ -168,8 +170,13 @@ def prefix_cache_replay(window: int, ops):
                 cached.add(toks[:p + 1])
             for p in win:
                 refs[toks[:p + 1]] = refs.get(toks[:p + 1], 0) + 1
+            inserted[toks] = inserted.get(toks, 0) + 1
         elif kind == "release":
-            assert toks[:n] in cached or n == 0, "release of a sequence that is not cached"
+            if n == 0:
+                continue
+            if inserted.get(toks, 0) == 0:
+                raise ValueError("release of a sequence with no insert left to undo")
+            inserted[toks] -= 1
             for p in win:
                 key = toks[:p + 1]
                 refs[key] = max(0, refs.get(key, 0) - 1)

@@ -147,3 +147,42 @@ def test_errors():
     assert e.value.code == hs.HSWA_ERR_INVALID_ARG
     assert t.match([]) == (0, 0)
     assert t.evict_swa([5, 6], 0, 10) == 0  # nothing cached on that path
+
+
+def test_release_needs_an_insert_of_exactly_those_tokens():
+    # A release undoes one insert of the same tokens. Releasing a cached prefix that was never
+    # inserted on its own, or releasing one insert twice, would take window counts that belong
+    # to other cached sequences; both are rejected and leave the state unchanged.
+    W = 4
+    A = list(range(1, 11))
+    t = hs.PrefixTree(W)
+    t.insert(A)
+    t.insert(A[:6])
+    for bad in (A[:8], A[:3], A + [99]):
+        with pytest.raises(hs.HswaError) as e:
+            t.release(bad)
+        assert e.value.code == hs.HSWA_ERR_INVALID_ARG
+        with pytest.raises(ValueError):
+            oracle.prefix_cache_replay(W, [("insert", A), ("insert", A[:6]), ("release", bad)])
+    # the rejected releases changed nothing: both windows still count
+    assert t.match(A) == (10, 10)
+    assert t.match(A[:6]) == (6, 6)
+    t.release(A[:6])
+    with pytest.raises(hs.HswaError):
+        t.release(A[:6])  # its one insert is already undone
+    with pytest.raises(ValueError):
+        oracle.prefix_cache_replay(W, [("insert", A), ("insert", A[:6]), ("release", A[:6]),
+                                       ("release", A[:6])])
+    assert t.match(A[:6]) == (6, 0)
+    assert t.match(A) == (10, 10)
+    # two inserts of the same tokens take two releases
+    t.insert(A)
+    t.release(A)
+    assert t.match(A) == (10, 10)
+    t.release(A)
+    assert t.match(A) == (10, 0)
+    t.release([])  # the empty sequence: nothing to undo, accepted
+    ops = [("insert", A), ("insert", A[:6]), ("insert", A), ("release", A[:6]), ("release", A),
+           ("match", A), ("release", A), ("match", A), ("match", A[:6]), ("release", [])]
+    assert oracle.prefix_cache_replay(W, ops) == [(10, 10), (10, 0), (6, 0)]
+    t.close()
