@@ -37,6 +37,11 @@ import torch
 import synth
 
 METRIC = "SWA/full prefill TFLOP/s (% BF16 peak); hybrid decode KV GB/s (% HBM peak)"
+ATOL_MAX, ATOL_MEAN = 2e-2, 2e-3  # attention parity against the fp64 oracle (max-abs, mean-abs)
+
+
+def parity_ok(max_err, mean_err) -> bool:
+    return max_err is not None and max_err <= ATOL_MAX and mean_err <= ATOL_MEAN
 SEED = 20261202
 
 
@@ -147,6 +152,14 @@ def gen(tag, layer, seq, pos0, n, h, d, sigma, device):
 class SwaPrefill16k:
     """Mistral-shaped SWA prefill of one 16K chunk (B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128)."""
     name = "swa_prefill_16k_B2_W4096_Hq32_Hkv8_d128"
+
+    @staticmethod
+    def config(ws, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128):
+        """The config dict of this workload's JSON line (the same for both arms)."""
+        return {"workload": SwaPrefill16k.name, "B_per_gpu": B, "seq_len": N, "window": W, "Hq": Hq,
+                "Hkv": Hkv, "head_dim": d, "parallelism": f"independent batches x{ws}",
+                "step": "swa_prefill_fwd + kv_pool_append(ring commit)",
+                "l2": "inputs larger than L2 (Q 268 MB + K/V 134 MB + O 268 MB per step)"}
 
     def __init__(self, hs, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128, seq_offset=0):
         self.hs = hs
@@ -546,11 +559,12 @@ class DecodeBatch:
             ho.copy_(o, non_blocking=True)
 
     def check_sample(self, oracle):
-        """All rows of the two shortest sequences on the full layer and of two sequences on an SWA layer."""
+        """All rows of the two shortest sequences and of the longest one (the most splits to merge) on
+        the full layer, and of two sequences on an SWA layer."""
         lens, nq, Hq, Hkv, d, W = self.lens, self.nq, self.Hq, self.Hkv, self.d, self.W
         order = torch.argsort(lens)
         errs = []
-        for b in [int(order[0]), int(order[1])]:
+        for b in [int(order[0]), int(order[1]), int(order[-1])]:
             L = int(lens[b])
             k = gen(synth.TAG_K, self.full_layer, self.base + b, 0, L + nq, Hkv, d, 1.0, "cpu")
             v = gen(synth.TAG_V, self.full_layer, self.base + b, 0, L + nq, Hkv, d, 1.0, "cpu")
@@ -811,7 +825,7 @@ def run_reference(args, ws, rank):
     line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1000, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": SwaPrefill16k.name, "B": B, "N": N, "W": W, "Hq": Hq, "Hkv": Hkv, "head_dim": d},
+            "config": SwaPrefill16k.config(ws, B, N, W, Hq, Hkv, d),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": f"{n_rows} query rows x {Hq} heads at the end of sequence 0 (full W-key windows) per step"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -1004,10 +1018,7 @@ def main():
                       "l2": "inputs larger than L2 (tens of GB of K/V per step)"}
             kname = "hybrid_decode_fwd on the full layer (plan_kernel + decode_kernel<128,2> + merge_kernel)"
         else:
-            config = {"workload": wl.name, "B_per_gpu": wl.B, "seq_len": wl.N, "window": wl.W, "Hq": wl.Hq,
-                      "Hkv": wl.Hkv, "head_dim": wl.d, "parallelism": f"independent batches x{ws}",
-                      "step": "swa_prefill_fwd + kv_pool_append(ring commit)",
-                      "l2": "inputs larger than L2 (Q 268 MB + K/V 134 MB + O 268 MB per step)"}
+            config = SwaPrefill16k.config(ws, wl.B, wl.N, wl.W, wl.Hq, wl.Hkv, wl.d)
             kname = "prefill_kernel<128> (swa_prefill_fwd)"
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": ws,
@@ -1036,9 +1047,25 @@ def main():
                                 "(70 layers of Q plus the SWA chunks' K/V)")
         if sec:
             line["secondary"] = sec
+        bad = []
+        if not parity_ok(max_err, mean_err):
+            bad.append(wl.name)
+        for r in sec or []:
+            if "max_abs_err" in r and not parity_ok(r["max_abs_err"], r["mean_abs_err"]):
+                bad.append(r["workload"])
+            if r.get("bit_exact") is False:
+                bad.append(r["workload"])
+        line["parity"]["ok"] = not bad
+        if bad:
+            line["parity"]["failed"] = bad
         print(json.dumps(line), flush=True)
+    else:
+        bad = []
     if ws > 1:
         torch.distributed.destroy_process_group()
+    if bad:
+        sys.stderr.write(f"parity check failed against the oracle: {bad}\n")
+        sys.exit(1)
 
 
 if __name__ == "__main__":

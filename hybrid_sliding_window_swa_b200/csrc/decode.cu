@@ -641,22 +641,16 @@ __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
   }
 }
 
-int64_t max_items(int n_seqs, int Hkv, int window, int64_t max_ctx_len) {
-  int64_t cached = window > 0 ? (max_ctx_len < window ? max_ctx_len : window - 1) : max_ctx_len;
-  int64_t nsp = (cached + SPLIT - 1) / SPLIT;
-  if (nsp < 1) nsp = 1;
-  return (int64_t)n_seqs * Hkv * nsp;
+// Largest split count of any sequence for these arguments.
+int64_t max_splits(int window, int64_t max_ctx_len) {
+  const int64_t cached = window > 0 ? (max_ctx_len < window ? max_ctx_len : window - 1) : max_ctx_len;
+  const int64_t nsp = (cached + SPLIT - 1) / SPLIT;
+  return nsp < 1 ? 1 : nsp;
 }
 
 template <int D, int MT>
-int launch_t(DecParams& p, int n_items_max, cudaStream_t stream) {
+int launch_t(DecParams& p, int n_items_max, int sms, size_t merge_smem, cudaStream_t stream) {
   using SM = DecSmem<D, MT>;
-  static int sms = 0;
-  if (!sms) {
-    int dev;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
   plan_kernel<<<1, 1024, 0, stream>>>(p);
   cudaFuncSetAttribute(decode_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::BYTES);
   int per_sm = 2;
@@ -664,14 +658,10 @@ int launch_t(DecParams& p, int n_items_max, cudaStream_t stream) {
   if (grid > n_items_max) grid = n_items_max;
   if (grid < 1) grid = 1;
   decode_kernel<D, MT><<<grid, DEC_THREADS, SM::BYTES, stream>>>(p);
-  {
-    const int64_t max_nsp = max_items(p.n_seqs, p.Hkv, p.window, p.max_ctx_len) / ((int64_t)p.n_seqs * p.Hkv);
-    if (max_nsp > 1) {
-      const size_t msm = ((size_t)max_nsp + 1) * p.R * sizeof(float);
-      if (msm > 48 * 1024)
-        cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msm);
-      merge_kernel<D><<<p.n_seqs * p.Hkv, 256, msm, stream>>>(p);
-    }
+  if (merge_smem > 0) {
+    if (merge_smem > 48 * 1024)
+      cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)merge_smem);
+    merge_kernel<D><<<p.n_seqs * p.Hkv, 256, merge_smem, stream>>>(p);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -686,8 +676,16 @@ int launch_t(DecParams& p, int n_items_max, cudaStream_t stream) {
 size_t decode_workspace_bytes(int n_seqs, int n_qt, int Hq, int Hkv, int d, int window, int64_t max_ctx_len) {
   const int G = Hq / Hkv;
   const int rows = n_qt * G;
-  WsLayout L(n_seqs, rows, d, max_items(n_seqs, Hkv, window, max_ctx_len));
+  WsLayout L(n_seqs, rows, d, (int64_t)n_seqs * Hkv * max_splits(window, max_ctx_len));
   return L.bytes;
+}
+
+size_t decode_merge_smem_bytes(int n_seqs, int n_qt, int Hq, int Hkv, int window, int64_t max_ctx_len) {
+  (void)n_seqs;
+  const int64_t nsp = max_splits(window, max_ctx_len);
+  if (nsp <= 1) return 0;
+  // [nsp][R] scale factors and [R] inverse denominators
+  return (size_t)(nsp + 1) * (size_t)(n_qt * (Hq / Hkv)) * sizeof(float);
 }
 
 int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
@@ -720,7 +718,7 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)Lc.d));
   p.ws = static_cast<uint8_t*>(Lc.workspace);
   p.err = pool->err;
-  const int64_t mi = max_items(p.n_seqs, p.Hkv, p.window, p.max_ctx_len);
+  const int64_t mi = (int64_t)p.n_seqs * p.Hkv * max_splits(p.window, p.max_ctx_len);
   WsLayout WL(p.n_seqs, p.R, Lc.d, mi);
   p.part_off = WL.part_off;
   p.part_bytes = WL.part_bytes_per_item;
@@ -730,10 +728,12 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
     return HSWA_ERR_UNSUPPORTED_SHAPE;
   }
   const int nmax = mi > 0x7fffffff ? 0x7fffffff : (int)mi;
+  const size_t msm = decode_merge_smem_bytes(p.n_seqs, p.n_qt, p.Hq, p.Hkv, p.window, p.max_ctx_len);
+  const int sms = pool->sms;
   if (Lc.d == 128) {
-    return p.R <= 16 ? launch_t<128, 1>(p, nmax, stream) : launch_t<128, 2>(p, nmax, stream);
+    return p.R <= 16 ? launch_t<128, 1>(p, nmax, sms, msm, stream) : launch_t<128, 2>(p, nmax, sms, msm, stream);
   }
-  return p.R <= 16 ? launch_t<64, 1>(p, nmax, stream) : launch_t<64, 2>(p, nmax, stream);
+  return p.R <= 16 ? launch_t<64, 1>(p, nmax, sms, msm, stream) : launch_t<64, 2>(p, nmax, sms, msm, stream);
 }
 
 }  // namespace hswa
@@ -779,68 +779,21 @@ extern "C" int hybrid_decode_fwd_noalloc(hswa_pool* pool, int layer, const hswa_
                                          const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq,
                                          const int64_t* ctx_len, int64_t max_ctx_len, const int32_t* seq_ids,
                                          const int32_t* page_table, int pt_stride, int n_q_heads, void* stream) {
-  using hswa::set_error;
-  if (!pool) {
-    set_error("hybrid_decode_fwd_noalloc: null pool");
-    return HSWA_ERR_INVALID_ARG;
-  }
-  const hswa_pool_desc& D = pool->desc;
-  if (layer < 0 || layer >= D.n_swa_layers + D.n_full_layers) {
-    set_error("hybrid_decode_fwd_noalloc: layer %d out of range", layer);
-    return HSWA_ERR_INVALID_ARG;
-  }
-  const int hkv = D.n_kv_heads;
-  if (n_q_heads < 1 || n_q_heads % hkv != 0 || n_q_heads / hkv > 16) {
-    set_error("hybrid_decode_fwd_noalloc: n_q_heads %d must be a positive multiple of n_kv_heads %d (ratio <= 16)",
-              n_q_heads, hkv);
-    return HSWA_ERR_UNSUPPORTED_SHAPE;
-  }
-  if (n_seqs < 0 || n_q_per_seq < 1 || n_q_per_seq > 8 || max_ctx_len < 0) {
-    set_error("hybrid_decode_fwd_noalloc: bad sizes (n_q_per_seq must be 1..8)");
-    return HSWA_ERR_INVALID_ARG;
-  }
-  if (max_ctx_len > 0x7fffffffLL - 4096) {
-    set_error("hybrid_decode_fwd_noalloc: positions must stay below 2^31");
-    return HSWA_ERR_UNSUPPORTED_SHAPE;
-  }
-  if (n_seqs == 0) return HSWA_OK;
-  const bool is_swa = layer < D.n_swa_layers;
-  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
-  if (!q || !k_new || !v_new || !o || !ctx_len || misaligned(q) || misaligned(k_new) || misaligned(v_new) ||
-      misaligned(o) || (is_swa && !seq_ids) || (!is_swa && (!page_table || pt_stride < 1))) {
-    set_error("hybrid_decode_fwd_noalloc: missing or misaligned device pointer");
-    return HSWA_ERR_INVALID_ARG;
-  }
-  const size_t need = hswa::decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, hkv, D.head_dim,
-                                                   is_swa ? D.window : 0, max_ctx_len);
+  hswa::DecodeLaunch L;
+  size_t need = 0;
+  // the same argument checks as hybrid_decode_fwd (including that the pool's device is current)
+  int rc = hswa::prepare_decode(pool, "hybrid_decode_fwd_noalloc", layer, q, k_new, v_new, o, n_seqs, n_q_per_seq,
+                                ctx_len, max_ctx_len, seq_ids, page_table, pt_stride, n_q_heads, &L, &need);
+  if (rc || L.n_seqs == 0) return rc;
   if (need > (size_t)HSWA_NOALLOC_SCRATCH_BYTES) {
-    set_error("hybrid_decode_fwd_noalloc: this call needs %zu bytes of scratch but the built-in array holds %zu; "
-              "use hybrid_decode_fwd with a caller-provided workspace",
-              need, (size_t)HSWA_NOALLOC_SCRATCH_BYTES);
+    hswa::set_error("hybrid_decode_fwd_noalloc: this call needs %zu bytes of scratch but the built-in array holds "
+                    "%zu; use hybrid_decode_fwd with a caller-provided workspace",
+                    need, (size_t)HSWA_NOALLOC_SCRATCH_BYTES);
     return HSWA_ERR_OUT_OF_MEMORY;
   }
   void* scratch = nullptr;
-  int rc = noalloc_scratch(&scratch);
+  rc = noalloc_scratch(&scratch);
   if (rc) return rc;
-  hswa::DecodeLaunch L{};
-  L.n_seqs = n_seqs;
-  L.n_qt = n_q_per_seq;
-  L.Hq = n_q_heads;
-  L.Hkv = hkv;
-  L.d = D.head_dim;
-  L.window = is_swa ? D.window : 0;
-  L.q = q;
-  L.k_new = k_new;
-  L.v_new = v_new;
-  L.o = o;
-  L.ctx_len = ctx_len;
-  L.max_ctx_len = max_ctx_len;
-  L.seq_ids = seq_ids;
-  L.page_table = page_table;
-  L.pt_stride = pt_stride;
-  L.pool = pool;
-  L.ring_layer = is_swa ? layer : 0;
-  L.full_layer = is_swa ? 0 : layer - D.n_swa_layers;
   L.workspace = scratch;
   L.ws_bytes = (size_t)HSWA_NOALLOC_SCRATCH_BYTES;
   return hswa::launch_decode(L, static_cast<cudaStream_t>(stream));

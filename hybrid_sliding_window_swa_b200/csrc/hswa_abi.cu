@@ -68,6 +68,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
 
 static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+int check_device(const hswa_pool* pool, const char* who) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_error("%s: no current CUDA device: %s", who, cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  if (dev != pool->device) {
+    set_error("%s: the pool lives on device %d but device %d is current", who, pool->device, dev);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  return HSWA_OK;
+}
+
 static int check_desc(const hswa_pool_desc* d) {
   if (!d) {
     set_error("null pool descriptor");
@@ -149,7 +163,15 @@ int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa
     return HSWA_ERR_OUT_OF_MEMORY;
   }
   p->desc = *desc;
-  cudaGetDevice(&p->device);
+  cudaError_t de = cudaGetDevice(&p->device);
+  if (de == cudaSuccess) de = cudaDeviceGetAttribute(&p->sms, cudaDevAttrMultiProcessorCount, p->device);
+  if (de == cudaSuccess)
+    de = cudaDeviceGetAttribute(&p->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device);
+  if (de != cudaSuccess || p->sms < 1) {
+    set_error("kv_pool_create: querying the current device failed: %s", cudaGetErrorString(de));
+    delete p;
+    return HSWA_ERR_CUDA;
+  }
   p->base = static_cast<uint8_t*>(dev_mem);
   p->bytes_swa = swa;
   p->bytes_full = full;
@@ -225,6 +247,7 @@ int kv_pool_append(hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_id
     set_error("kv_pool_append: negative sizes");
     return HSWA_ERR_INVALID_ARG;
   }
+  if (int rc = check_device(pool, "kv_pool_append")) return rc;
   if (n_seqs == 0 || n_tok == 0) return HSWA_OK;
   const bool is_swa = layer < D.n_swa_layers;
   if (!k || !v || !start_pos || !aligned16(k) || !aligned16(v) || (is_swa && !seq_ids) ||
@@ -265,6 +288,7 @@ int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_b
   }
   int rc = check_heads(pool, n_q_heads);
   if (rc) return rc;
+  if ((rc = check_device(pool, "swa_prefill_fwd"))) return rc;
   if (B < 0 || n_q < 0 || B > 65535) {
     set_error("swa_prefill_fwd: bad B or n_q");
     return HSWA_ERR_INVALID_ARG;
@@ -311,6 +335,7 @@ int full_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, hswa_bf16* 
   }
   int rc = check_heads(pool, n_q_heads);
   if (rc) return rc;
+  if ((rc = check_device(pool, "full_prefill_fwd"))) return rc;
   if (B < 0 || n_q < 0 || B > 65535) {
     set_error("full_prefill_fwd: bad B or n_q");
     return HSWA_ERR_INVALID_ARG;
@@ -354,61 +379,94 @@ int hybrid_decode_workspace_size(const hswa_pool* pool, int n_seqs, int n_q_per_
   return HSWA_OK;
 }
 
-int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
-                      const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq, const int64_t* ctx_len,
-                      int64_t max_ctx_len, const int32_t* seq_ids, const int32_t* page_table, int pt_stride,
-                      int n_q_heads, void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace hswa {
+
+int prepare_decode(hswa_pool* pool, const char* who, int layer, const uint16_t* q, const uint16_t* k_new,
+                   const uint16_t* v_new, uint16_t* o, int n_seqs, int n_q_per_seq, const int64_t* ctx_len,
+                   int64_t max_ctx_len, const int32_t* seq_ids, const int32_t* page_table, int pt_stride,
+                   int n_q_heads, DecodeLaunch* L, size_t* need) {
   if (!pool) {
-    set_error("hybrid_decode_fwd: null pool");
+    set_error("%s: null pool", who);
     return HSWA_ERR_INVALID_ARG;
   }
   const hswa_pool_desc& D = pool->desc;
   if (layer < 0 || layer >= D.n_swa_layers + D.n_full_layers) {
-    set_error("hybrid_decode_fwd: layer %d out of range", layer);
+    set_error("%s: layer %d out of range", who, layer);
     return HSWA_ERR_INVALID_ARG;
   }
   int rc = check_heads(pool, n_q_heads);
   if (rc) return rc;
   if (n_seqs < 0 || n_q_per_seq < 1 || n_q_per_seq > 8 || max_ctx_len < 0) {
-    set_error("hybrid_decode_fwd: bad sizes (n_q_per_seq must be 1..8)");
+    set_error("%s: bad sizes (n_q_per_seq must be 1..8)", who);
     return HSWA_ERR_INVALID_ARG;
   }
   if (max_ctx_len > 0x7fffffffLL - 4096) {
-    set_error("hybrid_decode_fwd: positions must stay below 2^31");
+    set_error("%s: positions must stay below 2^31", who);
     return HSWA_ERR_UNSUPPORTED_SHAPE;
   }
+  const int rows = n_q_per_seq * (n_q_heads / D.n_kv_heads);
+  if (rows > 32) {
+    set_error("%s: n_q_per_seq * (n_q_heads / n_kv_heads) = %d rows per KV head; at most 32 supported", who, rows);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if ((rc = check_device(pool, who))) return rc;
+  *L = DecodeLaunch{};
+  *need = 0;
   if (n_seqs == 0) return HSWA_OK;
   const bool is_swa = layer < D.n_swa_layers;
   if (!q || !k_new || !v_new || !o || !ctx_len || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
       !aligned16(o) || (is_swa && !seq_ids) || (!is_swa && (!page_table || pt_stride < 1))) {
-    set_error("hybrid_decode_fwd: missing or misaligned device pointer");
+    set_error("%s: missing or misaligned device pointer", who);
     return HSWA_ERR_INVALID_ARG;
   }
-  const size_t need = decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, D.n_kv_heads, D.head_dim,
-                                             is_swa ? D.window : 0, max_ctx_len);
+  const int window = is_swa ? D.window : 0;
+  const size_t msm = decode_merge_smem_bytes(n_seqs, n_q_per_seq, n_q_heads, D.n_kv_heads, window, max_ctx_len);
+  if (msm > (size_t)pool->smem_optin) {
+    set_error("%s: max_ctx_len %lld gives %zu bytes of split-merge shared memory; this device allows %d", who,
+              (long long)max_ctx_len, msm, pool->smem_optin);
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  *need = decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, D.n_kv_heads, D.head_dim, window, max_ctx_len);
+  L->n_seqs = n_seqs;
+  L->n_qt = n_q_per_seq;
+  L->Hq = n_q_heads;
+  L->Hkv = D.n_kv_heads;
+  L->d = D.head_dim;
+  L->window = window;
+  L->q = q;
+  L->k_new = k_new;
+  L->v_new = v_new;
+  L->o = o;
+  L->ctx_len = ctx_len;
+  L->max_ctx_len = max_ctx_len;
+  L->seq_ids = seq_ids;
+  L->page_table = page_table;
+  L->pt_stride = pt_stride;
+  L->pool = pool;
+  L->ring_layer = is_swa ? layer : 0;
+  L->full_layer = is_swa ? 0 : layer - D.n_swa_layers;
+  return HSWA_OK;
+}
+
+}  // namespace hswa
+
+extern "C" {
+
+int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
+                      const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq, const int64_t* ctx_len,
+                      int64_t max_ctx_len, const int32_t* seq_ids, const int32_t* page_table, int pt_stride,
+                      int n_q_heads, void* workspace, size_t ws_bytes, void* stream) {
+  DecodeLaunch L;
+  size_t need = 0;
+  int rc = prepare_decode(pool, "hybrid_decode_fwd", layer, q, k_new, v_new, o, n_seqs, n_q_per_seq, ctx_len,
+                          max_ctx_len, seq_ids, page_table, pt_stride, n_q_heads, &L, &need);
+  if (rc || L.n_seqs == 0) return rc;
   if (ws_bytes < need || (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)))) {
     set_error("hybrid_decode_fwd: workspace of %zu bytes (256-aligned) needed, %zu given", need, ws_bytes);
     return HSWA_ERR_INVALID_ARG;
   }
-  DecodeLaunch L{};
-  L.n_seqs = n_seqs;
-  L.n_qt = n_q_per_seq;
-  L.Hq = n_q_heads;
-  L.Hkv = D.n_kv_heads;
-  L.d = D.head_dim;
-  L.window = is_swa ? D.window : 0;
-  L.q = q;
-  L.k_new = k_new;
-  L.v_new = v_new;
-  L.o = o;
-  L.ctx_len = ctx_len;
-  L.max_ctx_len = max_ctx_len;
-  L.seq_ids = seq_ids;
-  L.page_table = page_table;
-  L.pt_stride = pt_stride;
-  L.pool = pool;
-  L.ring_layer = is_swa ? layer : 0;
-  L.full_layer = is_swa ? 0 : layer - D.n_swa_layers;
   L.workspace = workspace;
   L.ws_bytes = ws_bytes;
   return launch_decode(L, static_cast<cudaStream_t>(stream));
@@ -434,6 +492,7 @@ int hswa_selftest_wait_timeout(hswa_pool* pool, int64_t limit_ns, void* stream) 
     set_error("hswa_selftest_wait_timeout: a pool and a limit of 1 ms .. 2 s are required");
     return HSWA_ERR_INVALID_ARG;
   }
+  if (int rc = check_device(pool, "hswa_selftest_wait_timeout")) return rc;
   return launch_selftest_wait(pool->err, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream));
 }
 
@@ -442,6 +501,7 @@ int hswa_pool_check_error(hswa_pool* pool, int* device_code) {
     set_error("hswa_pool_check_error: null argument");
     return HSWA_ERR_INVALID_ARG;
   }
+  if (int rc = check_device(pool, "hswa_pool_check_error")) return rc;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     set_error("hswa_pool_check_error: device synchronisation failed: %s", cudaGetErrorString(e));

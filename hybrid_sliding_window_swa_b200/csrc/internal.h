@@ -9,7 +9,9 @@
 
 struct hswa_pool {
   hswa_pool_desc desc;
-  int device;
+  int device;        // the CUDA device current at kv_pool_create; every call must run with it current
+  int sms;           // its multiprocessor count
+  int smem_optin;    // its largest opt-in shared memory per block (bytes)
   uint8_t* base;
   size_t bytes_swa, bytes_full;
   uint16_t* ring_k;  // [max_seqs][n_swa][Hkv][W][d]
@@ -27,6 +29,10 @@ namespace hswa {
 
 // Thread-local error message of the ABI layer.
 void set_error(const char* fmt, ...);
+
+// HSWA_OK when the calling thread's current CUDA device is the pool's device; otherwise
+// HSWA_ERR_INVALID_ARG with a message naming `who` (nothing may be launched for the call).
+int check_device(const hswa_pool* pool, const char* who);
 
 // Encode a 2-5 dimensional bf16 tiled tensor map with 128-byte swizzle.
 // dims/strides: innermost first; strides in bytes for dims 1.. (dim 0 is contiguous).
@@ -83,6 +89,16 @@ struct DecodeLaunch {
 };
 
 size_t decode_workspace_bytes(int n_seqs, int n_qt, int Hq, int Hkv, int d, int window, int64_t max_ctx_len);
+// Dynamic shared memory of the split merge for these arguments (0 when no sequence can have two splits).
+size_t decode_merge_smem_bytes(int n_seqs, int n_qt, int Hq, int Hkv, int window, int64_t max_ctx_len);
+
+// Argument checks shared by hybrid_decode_fwd and hybrid_decode_fwd_noalloc (messages name `who`).
+// On HSWA_OK, *L is filled except for workspace/ws_bytes and *need is the scratch the call uses;
+// L->n_seqs == 0 means there is nothing to launch.
+int prepare_decode(hswa_pool* pool, const char* who, int layer, const uint16_t* q, const uint16_t* k_new,
+                   const uint16_t* v_new, uint16_t* o, int n_seqs, int n_q_per_seq, const int64_t* ctx_len,
+                   int64_t max_ctx_len, const int32_t* seq_ids, const int32_t* page_table, int pt_stride,
+                   int n_q_heads, DecodeLaunch* L, size_t* need);
 int launch_decode(const DecodeLaunch& L, cudaStream_t stream);
 
 }  // namespace hswa

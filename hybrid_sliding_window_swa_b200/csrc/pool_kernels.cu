@@ -68,8 +68,7 @@ int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* s
   const bool is_swa = layer < D.n_swa_layers;
   const int64_t total = (int64_t)n_seqs * n_tok * D.n_kv_heads * (D.head_dim / 8);
   if (total == 0) return HSWA_OK;
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, pool->device);
+  const int sms = pool->sms;
   const int64_t want = (total + 255) / 256;
   const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
   uint16_t* dk = is_swa ? pool->ring_k : pool->page_k;

@@ -555,9 +555,7 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
     return HSWA_ERR_UNSUPPORTED_SHAPE;
   }
   p.n_units = (int)units;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = pool->sms;
   const int grid = p.n_units < sms ? p.n_units : sms;
 
   const CUtensorMap& rk = pool->ring_tma ? pool->tm_ring_k : Lc.tm_k;

@@ -96,3 +96,39 @@ def test_ctx_len_above_declared_max_is_reported():
     pt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
     hs.hybrid_decode_fwd(pool, 0, q, q, q, torch.tensor([200], device="cuda"), 100, ws, page_table=pt)
     assert hs.hswa_pool_check_error(pool) == hs.HSWA_ERR_DEVICE_BOUNDS
+
+
+def test_context_too_long_for_the_split_merge_is_rejected_before_launch():
+    # max_ctx_len near 2^31 means ~262K splits of one sequence: their merge factors need far more
+    # shared memory than a block may use, so both entry points refuse before launching anything
+    import ctypes
+    desc = hs.PoolDesc(n_swa_layers=0, n_full_layers=1, window=128, n_kv_heads=8, head_dim=128, max_seqs=1,
+                       pages_per_full_layer=4)
+    pool = hs.kv_pool_create(desc)
+    q = torch.zeros(1, 4, 64, 128, dtype=torch.bfloat16, device="cuda")
+    kn = torch.zeros(1, 4, 8, 128, dtype=torch.bfloat16, device="cuda")
+    ctx = torch.zeros(1, dtype=torch.int64, device="cuda")
+    pt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    lib = hs.load_library()
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())
+    big = (1 << 31) - 8192
+    rc = lib.hybrid_decode_fwd(pool.handle, 0, vp(q), vp(kn), vp(kn), vp(q), 1, 4, vp(ctx), big, None, vp(pt), 4, 64,
+                               None, 0, None)
+    assert rc == hs.HSWA_ERR_UNSUPPORTED_SHAPE and "shared memory" in lib.hswa_last_error().decode()
+    rc = lib.hybrid_decode_fwd_noalloc(pool.handle, 0, vp(q), vp(kn), vp(kn), vp(q), 1, 4, vp(ctx), big, None,
+                                       vp(pt), 4, 64, None)
+    assert rc == hs.HSWA_ERR_UNSUPPORTED_SHAPE and "shared memory" in lib.hswa_last_error().decode()
+    assert hs.hswa_pool_check_error(pool) == 0
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two GPUs")
+def test_calls_with_another_device_current_are_rejected():
+    desc = hs.PoolDesc(n_swa_layers=1, n_full_layers=0, window=128, n_kv_heads=1, head_dim=64, max_seqs=1,
+                       pages_per_full_layer=0)
+    with torch.cuda.device(0):
+        pool = hs.kv_pool_create(desc, device="cuda:0")
+        q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16, device="cuda:0")
+    with torch.cuda.device(1):
+        with pytest.raises(hs.HswaError) as e:
+            hs.swa_prefill_fwd(pool, 0, q, q, q)
+        assert e.value.code == hs.HSWA_ERR_INVALID_ARG and "device" in str(e.value)

@@ -15,6 +15,7 @@ import pytest
 import torch
 
 import hybrid_sliding_window_swa_b200 as hs
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -99,6 +100,16 @@ def test_noalloc_matches_workspace_decode_on_two_calls_in_a_row():
             torch.cuda.synchronize()
             assert hs.hswa_pool_check_error(pool) == 0
             _check_close(out, ref, f"call {call} layer {layer}")
+            # and directly against the fp64 oracle, on inputs regenerated on the CPU
+            d, W, hq, hkv, n_qt = c["d"], c["window"], c["hq"], c["hkv"], c["n_qt"]
+            for b, L in enumerate(c["lens"]):
+                base = max(0, L - W + 1) if layer == 0 else 0
+                kk = _rows(c["seed"], synth.TAG_K, layer, b, base, L + n_qt - base, hkv, d)
+                vv = _rows(c["seed"], synth.TAG_V, layer, b, base, L + n_qt - base, hkv, d)
+                qq = _rows(c["seed"], synth.TAG_Q, layer, b, L, n_qt, hq, d)
+                want = oracle.attention(qq, L + np.arange(n_qt), kk, vv, W if layer == 0 else 0, key_base=base)
+                err = np.abs(out[b].float().cpu().double().numpy() - want)
+                assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, f"call {call} layer {layer} seq {b}"
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
