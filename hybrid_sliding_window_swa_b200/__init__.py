@@ -31,6 +31,7 @@ EXPORTED = [
     "window_safe_len", "hswa_pool_check_error", "hswa_last_error", "hybrid_decode_fwd_noalloc",
     "hswa_selftest_wait_timeout", "hswa_tree_create", "hswa_tree_destroy", "hswa_tree_insert",
     "hswa_tree_release", "hswa_tree_evict_swa", "hswa_tree_match", "hswa_tree_match_batch", "hswa_tree_stats",
+    "hswa_tree_match_slots", "kv_pool_gather_ring",
 ]
 
 # scratch bytes available to hybrid_decode_fwd_noalloc (HSWA_NOALLOC_SCRATCH_BYTES in hswa.h)
@@ -80,8 +81,10 @@ def load_library(path: str | None = None):
         "hswa_selftest_wait_timeout": [p, i64, p],
         "hswa_tree_create": [ctypes.c_int32, ctypes.POINTER(p)],
         "hswa_tree_destroy": [p],
-        "hswa_tree_insert": [p, p, i64, ctypes.POINTER(i64)],
-        "hswa_tree_release": [p, p, i64],
+        "hswa_tree_insert": [p, p, i64, ctypes.c_int32, ctypes.POINTER(i64)],
+        "hswa_tree_release": [p, p, i64, ctypes.c_int32],
+        "hswa_tree_match_slots": [p, p, i64, ctypes.POINTER(i64), ctypes.POINTER(i64), p],
+        "kv_pool_gather_ring": [p, i32, ctypes.c_int32, p, p],
         "hswa_tree_evict_swa": [p, p, i64, i64, i64, ctypes.POINTER(i64)],
         "hswa_tree_match": [p, p, i64, ctypes.POINTER(i64), ctypes.POINTER(i64)],
         "hswa_tree_match_batch": [p, p, p, ctypes.c_int32, p, p],
@@ -221,6 +224,13 @@ def kv_pool_append(pool: KVPool, layer: int, k: torch.Tensor, v: torch.Tensor, s
         _ptr(page_table, torch.int32, "page_table"), pt_stride, _stream(stream)))
 
 
+def kv_pool_gather_ring(pool: KVPool, layer: int, dst_seq: int, src_seq: torch.Tensor, stream=None):
+    """Assemble ring row dst_seq of layer ``layer`` slot by slot from the rows src_seq[s] (int32 [W]
+    on the device; -1 leaves a slot as it is)."""
+    _check(load_library().kv_pool_gather_ring(pool.handle, layer, dst_seq, _ptr(src_seq, torch.int32, "src_seq"),
+                                              _stream(stream)))
+
+
 def swa_prefill_fwd(pool: KVPool, layer: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     o: torch.Tensor | None = None, start_pos: torch.Tensor | None = None,
                     seq_ids: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -347,15 +357,16 @@ class PrefixTree:
         except Exception:
             pass
 
-    def insert(self, tokens) -> int:
+    def insert(self, tokens, owner: int = -1) -> int:
+        """Cache tokens for `owner` (the ring row holding its window, or -1); returns positions added."""
         a, ptr = _tokens(tokens)
         added = ctypes.c_int64()
-        _check(load_library().hswa_tree_insert(self.handle, ptr, a.size, ctypes.byref(added)))
+        _check(load_library().hswa_tree_insert(self.handle, ptr, a.size, owner, ctypes.byref(added)))
         return added.value
 
-    def release(self, tokens):
+    def release(self, tokens, owner: int = -1):
         a, ptr = _tokens(tokens)
-        _check(load_library().hswa_tree_release(self.handle, ptr, a.size))
+        _check(load_library().hswa_tree_release(self.handle, ptr, a.size, owner))
 
     def evict_swa(self, tokens, pos_lo: int, pos_hi: int) -> int:
         a, ptr = _tokens(tokens)
@@ -369,6 +380,17 @@ class PrefixTree:
         m, s = ctypes.c_int64(), ctypes.c_int64()
         _check(load_library().hswa_tree_match(self.handle, ptr, a.size, ctypes.byref(m), ctypes.byref(s)))
         return m.value, s.value
+
+    def match_slots(self, tokens):
+        """(match length, window-safe length L, int32 numpy [W]: per ring slot, the owner holding the
+        position of [max(0, L - W), L) in that slot, else -1)."""
+        import numpy as np
+        a, ptr = _tokens(tokens)
+        m, s = ctypes.c_int64(), ctypes.c_int64()
+        owners = np.full(self.window, -1, dtype=np.int32)
+        _check(load_library().hswa_tree_match_slots(self.handle, ptr, a.size, ctypes.byref(m), ctypes.byref(s),
+                                                    owners.ctypes.data_as(ctypes.c_void_p)))
+        return m.value, s.value, owners
 
     def match_batch(self, requests):
         """(match lengths, window-safe lengths) as int64 numpy arrays for a list of token sequences."""

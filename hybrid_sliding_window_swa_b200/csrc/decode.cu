@@ -15,7 +15,8 @@
 // blocks of K and V through a 3-stage cp.async pipeline; each warp takes 16 keys of a
 // block, computes S = Q K^T and O += P V with mma.sync (bf16 in, fp32 accumulate), and
 // keeps its own online-softmax state; the 4 warp states are merged through shared
-// memory at the end of the item. Items with one split write the output directly; the
+// memory at the end of the item. The CTAs take items in the order plan_kernel builds (length
+// buckets and longest first, see PlanView). Items with one split write the output directly; the
 // others write (m, l, O) partials that merge_kernel combines:
 //   o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
 #include <mutex>
@@ -39,20 +40,47 @@ static_assert(SPLIT % 64 == 0, "splits start on page boundaries");
 struct WsHeader {
   int counter;
   int total_items;
-  int pad[62];
+  int body_total;  // splits before each sequence's last one, summed over all sequences
+  int pad[61];
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace: header, the work-list plan (five int arrays over the sequences), then one
+// (m, l, O) partial per work item.
 struct WsLayout {
-  size_t prefix_off, part_off, part_bytes_per_item, bytes;
+  size_t part_off, part_bytes_per_item, bytes;
   __host__ __device__ WsLayout(int n_seqs, int rows, int d, int64_t max_items) {
-    prefix_off = sizeof(WsHeader);
-    part_off = align256(prefix_off + sizeof(int) * (size_t)(n_seqs + 1));
+    part_off = align256(sizeof(WsHeader) + sizeof(int) * (5 * (size_t)n_seqs + 1));
     part_bytes_per_item = (size_t)rows * (d + 2) * sizeof(float);
     bytes = part_off + part_bytes_per_item * (size_t)max_items;
   }
 };
+
+// The order in which the persistent CTAs take work (built by plan_kernel each call).
+// Every split of a sequence but its last covers exactly SPLIT cached keys ("body" splits); the
+// last one ("tail") holds the rest plus the new tokens. The work list is
+//   part A: the body splits, sequence by sequence, longest length bucket first
+//           (>= 256K tokens, 64K..256K, < 64K; stable within a bucket);
+//   part B: one tail split per sequence, in descending size classes of SPLIT/8 keys.
+// Heavy items start first and the step ends on the lightest ones, so the CTAs finish together.
+struct PlanView {
+  int* prefix;  // [n + 1] body splits before position pos of part A
+  int* order;   // [n] part-A position -> sequence
+  int* inv_a;   // [n] sequence -> part-A position
+  int* tail;    // [n] part-B position -> sequence
+  int* inv_b;   // [n] sequence -> part-B position
+  __device__ PlanView(uint8_t* ws, int n) {
+    prefix = reinterpret_cast<int*>(ws + sizeof(WsHeader));
+    order = prefix + n + 1;
+    inv_a = order + n;
+    tail = inv_a + n;
+    inv_b = tail + n;
+  }
+};
+
+constexpr int NCLS_A = 3;  // length buckets of part A
+constexpr int NCLS_B = 8;  // size classes of part B
 
 struct DecParams {
   int n_seqs, n_qt, Hq, Hkv, G, R, window;
@@ -97,19 +125,104 @@ __device__ __forceinline__ int64_t safe_len(const DecParams& p, int s) {
   return L;
 }
 
-// Prefix sums of the split counts; resets the work counter.
+// Length bucket of a sequence (part A order: higher first).
+__device__ __forceinline__ int class_a(int64_t L) { return L >= 262144 ? 2 : (L >= 65536 ? 1 : 0); }
+
+// Size class of a sequence's last split (part B order: higher first).
+__device__ __forceinline__ int class_b(const DecParams& p, int64_t L) {
+  const int64_t cached = L - dec_klo(p, L);
+  const int64_t tail = cached - (int64_t)(n_splits(p, L) - 1) * SPLIT;  // 0 .. SPLIT
+  const int c = (int)(tail / (SPLIT / NCLS_B));
+  return c < NCLS_B - 1 ? c : NCLS_B - 1;
+}
+
+// Builds the work list (see PlanView) and resets the work counter. One block of 1024 threads:
+// class totals, then a stable placement chunk by chunk (warp ballots give each thread its rank
+// among earlier threads of its class), then prefix sums of the body splits in part-A order.
 __global__ void __launch_bounds__(1024) plan_kernel(DecParams p) {
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
-  int* prefix = reinterpret_cast<int*>(p.ws + sizeof(WsHeader));
-  __shared__ int carry;
+  PlanView pv(p.ws, p.n_seqs);
+  constexpr int NC = NCLS_A + NCLS_B;
+  __shared__ int cnt[NC];      // sequences per class (classes 0..2: part A, 3..10: part B)
+  __shared__ int cur[NC];      // next position of each class
+  __shared__ int wcnt[NC][32]; // this chunk: per-warp counts, then exclusive per-warp offsets
+  __shared__ int chunk_tot[NC];
   __shared__ int warp_sums[32];
-  if (threadIdx.x == 0) carry = 0;
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid < NC) cnt[tid] = 0;
   __syncthreads();
   for (int base = 0; base < p.n_seqs; base += 1024) {
-    const int s = base + threadIdx.x;
-    int v = s < p.n_seqs ? n_splits(p, safe_len(p, s)) : 0;
-    // block-wide inclusive scan
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int s = base + tid;
+    if (s < p.n_seqs) {
+      const int64_t L = safe_len(p, s);
+      atomicAdd(&cnt[class_a(L)], 1);
+      atomicAdd(&cnt[NCLS_A + class_b(p, L)], 1);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int k = NCLS_A - 1; k >= 0; --k) {
+      cur[k] = acc;
+      acc += cnt[k];
+    }
+    acc = 0;
+    for (int k = NC - 1; k >= NCLS_A; --k) {
+      cur[k] = acc;
+      acc += cnt[k];
+    }
+  }
+  __syncthreads();
+  const unsigned lanes_below = (1u << lane) - 1u;
+  for (int base = 0; base < p.n_seqs; base += 1024) {
+    const int s = base + tid;
+    const bool live = s < p.n_seqs;
+    int ca = -1, cb = -1;
+    if (live) {
+      const int64_t L = safe_len(p, s);
+      ca = class_a(L);
+      cb = NCLS_A + class_b(p, L);
+    }
+    int rank_a = 0, rank_b = 0;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const unsigned m = __ballot_sync(0xffffffffu, k < NCLS_A ? ca == k : cb == k);
+      if (lane == 0) wcnt[k][w] = __popc(m);
+      if (k == ca) rank_a = __popc(m & lanes_below);
+      if (k == cb) rank_b = __popc(m & lanes_below);
+    }
+    __syncthreads();
+    if (w < NC) {  // warp k: exclusive scan of class k's per-warp counts
+      const int v = wcnt[w][lane];
+      int x = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, d);
+        if (lane >= d) x += y;
+      }
+      wcnt[w][lane] = x - v;
+      if (lane == 31) chunk_tot[w] = x;
+    }
+    __syncthreads();
+    if (live) {
+      const int pa = cur[ca] + wcnt[ca][w] + rank_a;
+      const int pb = cur[cb] + wcnt[cb][w] + rank_b;
+      pv.order[pa] = s;
+      pv.inv_a[s] = pa;
+      pv.tail[pb] = s;
+      pv.inv_b[s] = pb;
+    }
+    __syncthreads();
+    if (tid < NC) cur[tid] += chunk_tot[tid];
+    __syncthreads();
+  }
+  // prefix sums of the body splits over part-A positions (block-wide inclusive scan per chunk)
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < p.n_seqs; base += 1024) {
+    const int pos = base + tid;
+    const int v = pos < p.n_seqs ? n_splits(p, safe_len(p, pv.order[pos])) - 1 : 0;
     int x = v;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -119,24 +232,25 @@ __global__ void __launch_bounds__(1024) plan_kernel(DecParams p) {
     if (lane == 31) warp_sums[w] = x;
     __syncthreads();
     if (w == 0) {
-      int ws = warp_sums[lane];
+      int ws_ = warp_sums[lane];
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, ws, d);
-        if (lane >= d) ws += y;
+        const int y = __shfl_up_sync(0xffffffffu, ws_, d);
+        if (lane >= d) ws_ += y;
       }
-      warp_sums[lane] = ws;
+      warp_sums[lane] = ws_;
     }
     __syncthreads();
     const int incl = x + (w > 0 ? warp_sums[w - 1] : 0) + carry;
-    if (s < p.n_seqs) prefix[s + 1] = incl;
+    if (pos < p.n_seqs) pv.prefix[pos + 1] = incl;
     __syncthreads();
-    if (threadIdx.x == 1023) carry = incl;
+    if (tid == 1023) carry = incl;
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    prefix[0] = 0;
-    hdr->total_items = carry * p.Hkv;
+  if (tid == 0) {
+    pv.prefix[0] = 0;
+    hdr->body_total = carry;
+    hdr->total_items = (carry + p.n_seqs) * p.Hkv;
     hdr->counter = 0;
   }
 }
@@ -197,7 +311,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   WsHeader* hdr = reinterpret_cast<WsHeader*>(p.ws);
-  const int* prefix = reinterpret_cast<const int*>(p.ws + sizeof(WsHeader));
+  const PlanView pv(p.ws, p.n_seqs);
 
   if (read_error(p.err) != 0) return;
 
@@ -215,17 +329,25 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     if (item >= hdr->total_items) break;
     const int g = item % p.Hkv;
     const int sc = item / p.Hkv;
-    // sequence s: prefix[s] <= sc < prefix[s + 1]
-    int lo = 0, hi = p.n_seqs;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (prefix[mid] <= sc) lo = mid; else hi = mid;
+    int s, c;
+    if (sc < hdr->body_total) {
+      // part A: the position pos with prefix[pos] <= sc < prefix[pos + 1] (the largest such pos
+      // skips positions without body splits)
+      int lo = 0, hi = p.n_seqs;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pv.prefix[mid] <= sc) lo = mid; else hi = mid;
+      }
+      s = pv.order[lo];
+      c = sc - pv.prefix[lo];
+    } else {
+      s = pv.tail[sc - hdr->body_total];  // part B: the sequence's last split
+      c = -1;
     }
-    const int s = lo;
-    const int c = sc - prefix[s];
-    const int nsp = prefix[s + 1] - prefix[s];
-    const bool last = c == nsp - 1;
     const int L = (int)safe_len(p, s);
+    const int nsp = n_splits(p, L);
+    if (c < 0) c = nsp - 1;
+    const bool last = c == nsp - 1;
     const int klo = (int)dec_klo(p, L);
     const int a = klo + c * SPLIT;
     const int b = (a + SPLIT < L) ? a + SPLIT : L;
@@ -547,15 +669,20 @@ template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
   const int g = blockIdx.x % p.Hkv;
   const int s = blockIdx.x / p.Hkv;
-  const int* prefix = reinterpret_cast<const int*>(p.ws + sizeof(WsHeader));
-  const int c0 = prefix[s];
-  const int nsp = prefix[s + 1] - c0;
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(p.ws);
+  const PlanView pv(p.ws, p.n_seqs);
+  const int nsp = n_splits(p, safe_len(p, s));
   if (nsp <= 1) return;
   extern __shared__ float msh[];  // [nsp][R] scale factors, then [R] inverse denominators
   float* fac = msh;
   float* inv = msh + (size_t)nsp * p.R;
-  const uint8_t* part0 = p.ws + p.part_off + (size_t)(c0 * p.Hkv + g) * p.part_bytes;
-  const size_t split_stride = (size_t)p.Hkv * p.part_bytes;  // consecutive splits of this (s, g)
+  // partials of this (s, g): body splits are consecutive items of part A, the last split is in part B
+  const uint8_t* body0 = p.ws + p.part_off + ((size_t)pv.prefix[pv.inv_a[s]] * p.Hkv + g) * p.part_bytes;
+  const uint8_t* tailp = p.ws + p.part_off + ((size_t)(hdr->body_total + pv.inv_b[s]) * p.Hkv + g) * p.part_bytes;
+  const size_t split_stride = (size_t)p.Hkv * p.part_bytes;
+  auto split_part = [&](int c) -> const float* {
+    return reinterpret_cast<const float*>(c < nsp - 1 ? body0 + (size_t)c * split_stride : tailp);
+  };
   const int lane8 = threadIdx.x & 7;
   // rows padded to whole warps (4 rows of 8 threads per warp) so every shuffle has all 32 lanes
   const int r_pad = (p.R + 3) & ~3;
@@ -563,14 +690,14 @@ __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
     const bool live = r < p.R;
     float M = -INFINITY;
     for (int c = lane8; live && c < nsp; c += 8)
-      M = fmaxf(M, reinterpret_cast<const float*>(part0 + c * split_stride)[p.R * D + r]);
+      M = fmaxf(M, split_part(c)[p.R * D + r]);
     M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
     M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
     M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 4));
     const float Mo = M == -INFINITY ? 0.f : M;
     float den = 0.f;
     for (int c = lane8; live && c < nsp; c += 8) {
-      const float* part = reinterpret_cast<const float*>(part0 + c * split_stride);
+      const float* part = split_part(c);
       const float f = ex2_approx(part[p.R * D + r] - Mo);
       fac[c * p.R + r] = f;
       den += f * part[p.R * D + p.R + r];
@@ -597,8 +724,8 @@ __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
     }
     int c = 0;
     for (; c + 2 <= nsp; c += 2) {
-      const float* pa = reinterpret_cast<const float*>(part0 + c * split_stride);
-      const float* pb = reinterpret_cast<const float*>(part0 + (c + 1) * split_stride);
+      const float* pa = split_part(c);
+      const float* pb = split_part(c + 1);
       float4 va[4], vb[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -615,7 +742,7 @@ __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
       }
     }
     if (c < nsp) {
-      const float* pa = reinterpret_cast<const float*>(part0 + c * split_stride);
+      const float* pa = split_part(c);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float4 va = *reinterpret_cast<const float4*>(pa + it_r[u] * D + it_c[u]);

@@ -259,6 +259,24 @@ int kv_pool_append(hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_id
                        static_cast<cudaStream_t>(stream));
 }
 
+int kv_pool_gather_ring(hswa_pool* pool, int layer, int32_t dst_seq, const int32_t* src_seq, void* stream) {
+  if (!pool) {
+    set_error("kv_pool_gather_ring: null pool");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  if (layer < 0 || layer >= D.n_swa_layers) {
+    set_error("kv_pool_gather_ring: layer %d is not a sliding-window layer of this pool", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (dst_seq < 0 || dst_seq >= D.max_seqs || !src_seq) {
+    set_error("kv_pool_gather_ring: dst_seq %d outside [0, %d) or null src_seq", dst_seq, D.max_seqs);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (int rc = check_device(pool, "kv_pool_gather_ring")) return rc;
+  return launch_gather_ring(pool, layer, dst_seq, src_seq, static_cast<cudaStream_t>(stream));
+}
+
 static int build_q_map(CUtensorMap* m, const void* base, int B, int n_q, int H, int d) {
   const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)n_q, (uint64_t)B};
   const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)H * d * 2, (uint64_t)n_q * H * d * 2};

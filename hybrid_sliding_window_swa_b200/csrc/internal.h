@@ -43,6 +43,8 @@ int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* s
                   const int64_t* start_pos, int n_tok, const uint16_t* k, const uint16_t* v,
                   const int32_t* page_table, int pt_stride, cudaStream_t stream);
 
+int launch_gather_ring(const hswa_pool* pool, int layer, int dst, const int32_t* src, cudaStream_t stream);
+
 int launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t stream);
 
 int launch_window_safe_len(const int64_t* m, const int64_t* c, const uint32_t* valid, int W, int n_req,

@@ -92,6 +92,53 @@ int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* s
   return HSWA_OK;
 }
 
+// Ring row dst of one sliding-window layer, slot by slot from the rows src[s]: one thread moves 16
+// bytes of K and of V. Every ring keeps position p in slot p mod W, so a slot copied from another
+// row keeps its position.
+template <int D>
+__global__ void __launch_bounds__(256) gather_ring_kernel(uint16_t* __restrict__ ring_k, uint16_t* __restrict__ ring_v,
+                                                          const int32_t* __restrict__ src, int W, int Hkv, int n_swa,
+                                                          int layer, int max_seqs, int dst, int* err) {
+  constexpr int PER_ROW = D / 8;
+  const int64_t total = (int64_t)W * Hkv * PER_ROW;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(idx % PER_ROW);
+    const int64_t row = idx / PER_ROW;
+    const int g = (int)(row % Hkv);
+    const int slot = (int)(row / Hkv);
+    const int sq = src[slot];
+    if (sq < 0 || sq == dst) continue;
+    if (sq >= max_seqs) {
+      record_error(err, HSWA_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const int64_t from = ((((int64_t)sq * n_swa + layer) * Hkv + g) * W + slot) * D;
+    const int64_t to = ((((int64_t)dst * n_swa + layer) * Hkv + g) * W + slot) * D;
+    reinterpret_cast<uint4*>(ring_k + to)[c] = reinterpret_cast<const uint4*>(ring_k + from)[c];
+    reinterpret_cast<uint4*>(ring_v + to)[c] = reinterpret_cast<const uint4*>(ring_v + from)[c];
+  }
+}
+
+int launch_gather_ring(const hswa_pool* pool, int layer, int dst, const int32_t* src, cudaStream_t stream) {
+  const hswa_pool_desc& D = pool->desc;
+  const int64_t total = (int64_t)D.window * D.n_kv_heads * (D.head_dim / 8);
+  const int64_t want = (total + 255) / 256;
+  const int grid = (int)(want < (int64_t)pool->sms * 8 ? want : (int64_t)pool->sms * 8);
+  if (D.head_dim == 128)
+    gather_ring_kernel<128><<<grid, 256, 0, stream>>>(pool->ring_k, pool->ring_v, src, D.window, D.n_kv_heads,
+                                                       D.n_swa_layers, layer, D.max_seqs, dst, pool->err);
+  else
+    gather_ring_kernel<64><<<grid, 256, 0, stream>>>(pool->ring_k, pool->ring_v, src, D.window, D.n_kv_heads,
+                                                      D.n_swa_layers, layer, D.max_seqs, dst, pool->err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("kv_pool_gather_ring: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
 // One thread per request. With the ring holding positions [max(0, C-W), C):
 //  * C > W: the only resumable lengths are 0 and C (every other tail reaches a
 //    position older than C - W); C needs m >= C and all W slots valid.

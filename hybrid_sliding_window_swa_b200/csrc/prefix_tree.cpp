@@ -12,6 +12,12 @@
 //
 // With one cached sequence of length C this reduces to window_safe_len (a ring of W slots holding
 // positions [max(0, C - W), C)); here eviction is per position and cached sequences share prefixes.
+//
+// Every insert names an owner: the ring row where the caller keeps that sequence's sliding-window
+// KV. A position's holders are the owners whose window covers it and whose copy has not been
+// evicted since they were inserted; it holds sliding-window KV while it has a holder. A match can
+// report, for each ring slot of the resumed window, one holder's ring row, which is where that
+// position's KV can be copied from (slot = position mod W in every ring).
 #include <algorithm>
 #include <cstdint>
 #include <new>
@@ -26,19 +32,24 @@ void set_error(const char* fmt, ...);
 
 struct hswa_prefix_tree {
   // Path-compressed trie: node k holds a run of consecutive cached positions (its label) and,
-  // per position, the number of cached windows holding sliding-window KV there (0 after an
-  // eviction). Node 0 is the root with an empty label. A child is found by (node, first token).
+  // per position, the number of holders (owners whose window covers it and whose copy was not
+  // evicted since). Node 0 is the root with an empty label. A child is found by (node, first
+  // token). Each cached position has a stable id (pid0 + offset in the label; a split keeps the
+  // ids) that keys its holders and the owners of the inserts ending there.
   struct Node {
     int64_t pos0;                 // position of the label's first token
+    int64_t pid0;                 // id of the label's first position
     std::vector<int32_t> label;   // tokens at positions pos0 .. pos0 + label.size() - 1
-    std::vector<uint32_t> refs;   // per position of the label
-    std::vector<uint32_t> ends;   // per position: inserts (not yet released) that end there
+    std::vector<uint32_t> refs;   // per position of the label: number of holders
     std::vector<int32_t> kids;    // children (their first tokens key the lookup map)
   };
   int32_t window;
   std::vector<Node> nodes;
   std::unordered_map<uint64_t, int32_t> child;  // (node, first token of the child's label) -> child
+  std::unordered_map<int64_t, std::vector<int32_t>> holders;     // position id -> owners (refs > 0 only)
+  std::unordered_map<int64_t, std::vector<int32_t>> end_owners;  // position id -> owners of inserts ending there
   int64_t n_positions = 0;
+  int64_t next_pid = 0;
 
   static uint64_t key(int32_t n, int32_t t) { return ((uint64_t)(uint32_t)n << 32) | (uint32_t)t; }
   int32_t find(int32_t n, int32_t t) const {
@@ -102,7 +113,7 @@ int hswa_tree_create(int32_t window, hswa_prefix_tree** out) {
     return HSWA_ERR_OUT_OF_MEMORY;
   }
   t->window = window;
-  t->nodes.push_back(hswa_prefix_tree::Node{0, {}, {}, {}, {}});
+  t->nodes.push_back(hswa_prefix_tree::Node{0, 0, {}, {}, {}});
   *out = t;
   return HSWA_OK;
 }
@@ -112,7 +123,7 @@ int hswa_tree_destroy(hswa_prefix_tree* t) {
   return HSWA_OK;
 }
 
-int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int64_t* new_nodes) {
+int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int32_t owner, int64_t* new_nodes) {
   if (!t) {
     hswa::set_error("hswa_tree_insert: null tree");
     return HSWA_ERR_INVALID_ARG;
@@ -144,9 +155,9 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
         const int32_t tail = (int32_t)t->nodes.size();
         hswa_prefix_tree::Node tn;
         tn.pos0 = nd->pos0 + (int64_t)off;
+        tn.pid0 = nd->pid0 + (int64_t)off;
         tn.label.assign(nd->label.begin() + off, nd->label.end());
         tn.refs.assign(nd->refs.begin() + off, nd->refs.end());
-        tn.ends.assign(nd->ends.begin() + off, nd->ends.end());
         t->nodes.push_back(std::move(tn));
         nd = &t->nodes[node];  // the vector may have moved
         // the old children now hang under the tail node
@@ -160,7 +171,6 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
         t->child[hswa_prefix_tree::key(node, t->nodes[tail].label[0])] = tail;
         nd->label.resize(off);
         nd->refs.resize(off);
-        nd->ends.resize(off);
         break;
       }
       ++off;
@@ -174,10 +184,11 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
       const int32_t fresh = (int32_t)t->nodes.size();
       hswa_prefix_tree::Node fn;
       fn.pos0 = i;
+      fn.pid0 = t->next_pid;
       fn.label.assign(tokens + i, tokens + n);
       fn.refs.assign((size_t)(n - i), 0u);
-      fn.ends.assign((size_t)(n - i), 0u);
       t->nodes.push_back(std::move(fn));
+      t->next_pid += n - i;
       t->nodes[node].kids.push_back(fresh);
       t->child[hswa_prefix_tree::key(node, tokens[i])] = fresh;
       added = n - i;
@@ -187,41 +198,63 @@ int hswa_tree_insert(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int6
     hswa::set_error("hswa_tree_insert: out of host memory");
     return HSWA_ERR_OUT_OF_MEMORY;
   }
-  // 2. this sequence's window, its last W positions, now holds sliding-window KV, and one more
-  //    insert ends at its last position
+  // 2. this sequence's window, its last W positions, gains the owner as a holder, and one more
+  //    insert by this owner ends at its last position
   const int64_t win_lo = n > t->window ? n - t->window : 0;
-  t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
-    for (int64_t k = 0; k < len; ++k) {
-      if (pos + k >= win_lo) ++t->nodes[node].refs[off + (size_t)k];
-      if (pos + k == n - 1) ++t->nodes[node].ends[off + (size_t)k];
-    }
-  });
+  try {
+    t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+      hswa_prefix_tree::Node& nd = t->nodes[node];
+      for (int64_t k = 0; k < len; ++k) {
+        const int64_t pid = nd.pid0 + (int64_t)off + k;
+        if (pos + k >= win_lo) {
+          t->holders[pid].push_back(owner);
+          ++nd.refs[off + (size_t)k];
+        }
+        if (pos + k == n - 1) t->end_owners[pid].push_back(owner);
+      }
+    });
+  } catch (const std::bad_alloc&) {
+    hswa::set_error("hswa_tree_insert: out of host memory");
+    return HSWA_ERR_OUT_OF_MEMORY;
+  }
   if (new_nodes) *new_nodes = added;
   return HSWA_OK;
 }
 
-int hswa_tree_release(hswa_prefix_tree* t, const int32_t* tokens, int64_t n) {
+int hswa_tree_release(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int32_t owner) {
   if (!t) {
     hswa::set_error("hswa_tree_release: null tree");
     return HSWA_ERR_INVALID_ARG;
   }
   if (!check_tokens(tokens, n, "hswa_tree_release")) return HSWA_ERR_INVALID_ARG;
   if (n == 0) return HSWA_OK;  // the empty sequence holds nothing
-  // the sequence must be cached and at least one insert of exactly these tokens not yet released
-  uint32_t* end_count = nullptr;
+  // the sequence must be cached with an insert of exactly these tokens by this owner left
+  int64_t end_pid = -1;
   const int64_t m = t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
-    if (pos + len == n) end_count = &t->nodes[node].ends[off + (size_t)(len - 1)];
+    if (pos + len == n) end_pid = t->nodes[node].pid0 + (int64_t)off + len - 1;
   });
-  if (m != n || !end_count || *end_count == 0) {
-    hswa::set_error("hswa_tree_release: no insert of exactly this sequence is left to release");
+  auto eo = m == n ? t->end_owners.find(end_pid) : t->end_owners.end();
+  auto hit = eo == t->end_owners.end() ? std::vector<int32_t>::iterator()
+                                       : std::find(eo->second.begin(), eo->second.end(), owner);
+  if (eo == t->end_owners.end() || hit == eo->second.end()) {
+    hswa::set_error("hswa_tree_release: no insert of exactly this sequence by owner %d is left to release", owner);
     return HSWA_ERR_INVALID_ARG;
   }
-  --*end_count;
+  eo->second.erase(hit);
+  if (eo->second.empty()) t->end_owners.erase(eo);
+  // the owner stops holding its window (positions evicted since its insert no longer list it)
   const int64_t win_lo = n > t->window ? n - t->window : 0;
   t->walk(tokens, n, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    hswa_prefix_tree::Node& nd = t->nodes[node];
     for (int64_t k = 0; k < len; ++k) {
-      uint32_t& r = t->nodes[node].refs[off + (size_t)k];
-      if (pos + k >= win_lo && r > 0) --r;
+      if (pos + k < win_lo) continue;
+      auto h = t->holders.find(nd.pid0 + (int64_t)off + k);
+      if (h == t->holders.end()) continue;
+      auto o = std::find(h->second.begin(), h->second.end(), owner);
+      if (o == h->second.end()) continue;
+      h->second.erase(o);
+      nd.refs[off + (size_t)k] = (uint32_t)h->second.size();
+      if (h->second.empty()) t->holders.erase(h);
     }
   });
   return HSWA_OK;
@@ -236,10 +269,12 @@ int hswa_tree_evict_swa(hswa_prefix_tree* t, const int32_t* tokens, int64_t n, i
   if (!check_tokens(tokens, n, "hswa_tree_evict_swa")) return HSWA_ERR_INVALID_ARG;
   int64_t count = 0;
   t->walk(tokens, n < pos_hi ? n : (pos_hi > 0 ? pos_hi : 0), [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    hswa_prefix_tree::Node& nd = t->nodes[node];
     for (int64_t k = 0; k < len; ++k) {
-      uint32_t& r = t->nodes[node].refs[off + (size_t)k];
+      uint32_t& r = nd.refs[off + (size_t)k];
       if (pos + k >= pos_lo && r > 0) {
         r = 0;
+        t->holders.erase(nd.pid0 + (int64_t)off + k);
         ++count;
       }
     }
@@ -267,6 +302,28 @@ int hswa_tree_match(const hswa_prefix_tree* t, const int32_t* tokens, int64_t n,
   });
   *match_len = m;
   *safe_len = best;
+  return HSWA_OK;
+}
+
+int hswa_tree_match_slots(const hswa_prefix_tree* t, const int32_t* tokens, int64_t n, int64_t* match_len,
+                          int64_t* safe_len, int32_t* slot_owner) {
+  if (!slot_owner) {
+    hswa::set_error("hswa_tree_match_slots: null slot_owner");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const int rc = hswa_tree_match(t, tokens, n, match_len, safe_len);
+  if (rc) return rc;
+  const int64_t W = t->window, L = *safe_len;
+  for (int64_t s = 0; s < W; ++s) slot_owner[s] = -1;
+  const int64_t lo = L > W ? L - W : 0;
+  t->walk(tokens, L, [&](int32_t node, size_t off, int64_t pos, int64_t len) {
+    for (int64_t k = 0; k < len; ++k) {
+      if (pos + k < lo) continue;
+      auto h = t->holders.find(t->nodes[node].pid0 + (int64_t)off + k);
+      // every position of the safe tail has a holder; the most recent insert is reported
+      if (h != t->holders.end() && !h->second.empty()) slot_owner[(pos + k) % W] = h->second.back();
+    }
+  });
   return HSWA_OK;
 }
 

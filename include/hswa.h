@@ -119,6 +119,16 @@ HSWA_API int kv_pool_append(hswa_pool* pool, int layer, int n_seqs, const int32_
                    const int64_t* start_pos, int n_tok, const hswa_bf16* k, const hswa_bf16* v,
                    const int32_t* page_table, int pt_stride, void* stream);
 
+/* Assemble ring row dst_seq of sliding-window layer `layer` slot by slot: for each slot s with
+ * src_seq[s] >= 0, the K and V rows of slot s (all KV heads) are copied from ring row src_seq[s];
+ * slots with src_seq[s] = -1 or src_seq[s] = dst_seq are left as they are. Since every ring keeps
+ * position p in slot p mod W, this moves cached window positions held by other sequences' rings
+ * into the row of a request that resumes from a prefix-cache match (hswa_tree_match_slots gives
+ * src_seq). src_seq: device int32[W]. A source row outside [0, max_seqs) is skipped and recorded
+ * as HSWA_ERR_DEVICE_BOUNDS. Rows that are both a source and dst_seq must not be passed. */
+HSWA_API int kv_pool_gather_ring(hswa_pool* pool, int layer, int32_t dst_seq, const int32_t* src_seq,
+                                 void* stream);
+
 /* Causal sliding-window attention for one chunk of n_q new tokens per sequence
  * ("formal definition", eqs. (1)-(5), window W of the pool), on tensor cores.
  *  q, o    [B][n_q][n_q_heads][head_dim] bf16 (o written, rows in the chunk only)
@@ -208,9 +218,11 @@ HSWA_API int window_safe_len(const int64_t* match_len, const int64_t* cached_len
  * optimisation", section "KV cache redesign": a prefix-cache match is cut to the window-safe
  * length, since with sliding-window layers only part of a cached sequence's window KV may
  * survive). Each trie node is one cached position. Its full-attention KV is held while the node
- * exists; its sliding-window KV is held while at least one cached sequence's window (its last W
- * positions) covers it and it has not been evicted. With one cached sequence this is
- * window_safe_len with a per-position eviction mask; here cached sequences share prefixes.
+ * exists. Each insert names an owner: the ring row (sequence id of the pool) where the caller keeps
+ * that sequence's sliding-window KV, or -1. A position's holders are the owners whose window (their
+ * last W positions) covers it and whose copy has not been evicted since that insert; the position
+ * holds sliding-window KV while it has a holder. With one cached sequence this is window_safe_len
+ * with a per-position eviction mask; here cached sequences share prefixes.
  * Token ids are any int32 values. Calls on one tree are not thread-safe; the caller serialises
  * them. Errors: HSWA_ERR_INVALID_ARG for null pointers or negative lengths (nothing changes);
  * HSWA_ERR_OUT_OF_MEMORY when a host allocation fails during an insert, after which the tree
@@ -221,18 +233,19 @@ typedef struct hswa_prefix_tree hswa_prefix_tree;
 HSWA_API int hswa_tree_create(int32_t window, hswa_prefix_tree** out);
 HSWA_API int hswa_tree_destroy(hswa_prefix_tree* tree);
 
-/* Cache tokens[0..n): adds the missing positions and counts this sequence's window
- * [max(0, n-W), n) as holding sliding-window KV. *new_nodes (may be null) = positions added. */
-HSWA_API int hswa_tree_insert(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int64_t* new_nodes);
+/* Cache tokens[0..n) for `owner`: adds the missing positions and makes the owner a holder of this
+ * sequence's window [max(0, n-W), n). *new_nodes (may be null) = positions added. */
+HSWA_API int hswa_tree_insert(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int32_t owner,
+                              int64_t* new_nodes);
 
-/* Undo one hswa_tree_insert of the same tokens: its window stops counting (positions shared
- * with other cached windows stay held). HSWA_ERR_INVALID_ARG, with nothing changed, unless an
- * insert of exactly these tokens is left to undo (a cached prefix that was never inserted on its
- * own, or a second release of a single insert, is rejected). n = 0 is a no-op. */
-HSWA_API int hswa_tree_release(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n);
+/* Undo one hswa_tree_insert of the same tokens by the same owner: the owner stops holding that
+ * window (other holders keep their positions). HSWA_ERR_INVALID_ARG, with nothing changed, unless
+ * such an insert is left to undo (a cached prefix that was never inserted on its own, another
+ * owner's insert, or a second release of a single insert is rejected). n = 0 is a no-op. */
+HSWA_API int hswa_tree_release(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int32_t owner);
 
-/* Drop the sliding-window KV of positions [pos_lo, pos_hi) along the path tokens[0..n) (all
- * cached windows that cover them lose it); *evicted (may be null) = positions that held it. */
+/* Drop the sliding-window KV of positions [pos_lo, pos_hi) along the path tokens[0..n) (every
+ * holder loses it); *evicted (may be null) = positions that held it. */
 HSWA_API int hswa_tree_evict_swa(hswa_prefix_tree* tree, const int32_t* tokens, int64_t n, int64_t pos_lo,
                                  int64_t pos_hi, int64_t* evicted);
 
@@ -241,6 +254,13 @@ HSWA_API int hswa_tree_evict_swa(hswa_prefix_tree* tree, const int32_t* tokens, 
  * from. Exact integers. */
 HSWA_API int hswa_tree_match(const hswa_prefix_tree* tree, const int32_t* tokens, int64_t n,
                              int64_t* match_len, int64_t* safe_len);
+
+/* hswa_tree_match plus where the resumed window lives: slot_owner[W] (host memory) gets, for each
+ * position p in [max(0, L-W), L), at slot p mod W, the owner of the most recent insert that holds
+ * p; every other slot gets -1. kv_pool_gather_ring with these owners as sources assembles the
+ * request's ring for a prefill that starts at L. */
+HSWA_API int hswa_tree_match_slots(const hswa_prefix_tree* tree, const int32_t* tokens, int64_t n,
+                                   int64_t* match_len, int64_t* safe_len, int32_t* slot_owner);
 
 /* hswa_tree_match for n_req requests: request r is tokens[offsets[r] .. offsets[r+1]). */
 HSWA_API int hswa_tree_match_batch(const hswa_prefix_tree* tree, const int32_t* tokens, const int64_t* offsets,

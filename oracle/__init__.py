@@ -149,52 +149,65 @@ def prefix_cache_replay(window: int, ops):
     only part of a cached sequence's window KV may survive).
 
     State, by definition: a cached position is a token prefix (a tuple); every cached position
-    keeps its full-attention KV; its sliding-window KV is held while the number of cached
-    sequences whose last `window` positions include it is positive and it was not evicted since.
-    `ops` is a list of ("insert", tokens), ("release", tokens), ("evict", tokens, lo, hi) and
-    ("match", tokens); a release undoes one earlier insert of exactly the same tokens (ValueError
-    when none is left; the empty sequence is a no-op); returns, for each "match" in order,
-    (m, L): m = the longest cached prefix of tokens, L = max { L in [0, m] : every position in [max(0, L - window), L) holds its
-    sliding-window KV }. Quadratic in sequence length: for small cases only.
+    keeps its full-attention KV. Each insert names an owner (the ring row that keeps the
+    sequence's window KV; -1 when the caller does not say). A position's holders are the owners of
+    the inserts whose last `window` positions include it, counted once per insert, minus those
+    whose copy was evicted after their insert; it holds sliding-window KV while it has a holder.
+    `ops` is a list of ("insert", tokens[, owner]), ("release", tokens[, owner]),
+    ("evict", tokens, lo, hi), ("match", tokens) and ("match_slots", tokens). A release undoes one
+    earlier insert of exactly the same tokens by the same owner (ValueError when none is left; the
+    empty sequence is a no-op). Returns one result per match, in order: "match" gives (m, L),
+    m = the longest cached prefix of tokens, L = max { L in [0, m] : every position in
+    [max(0, L - window), L) holds sliding-window KV }; "match_slots" gives (m, L, slots) with
+    slots[s] = the set of holders of the position p of [max(0, L - window), L) with p mod window
+    = s (empty for the other slots). Quadratic in sequence length: for small cases only.
     """
     cached = set()
-    refs = {}
-    inserted = {}  # exact token tuple -> inserts not yet released
+    holders = {}   # token prefix -> list of owners (one entry per holding insert)
+    inserted = {}  # (exact token tuple, owner) -> inserts not yet released
     out = []
     for op in ops:
         kind, toks = op[0], tuple(int(t) for t in op[1])
         n = len(toks)
         win = range(max(0, n - window), n)
         if kind == "insert":
+            owner = int(op[2]) if len(op) > 2 else -1
             for p in range(n):
                 cached.add(toks[:p + 1])
             for p in win:
-                refs[toks[:p + 1]] = refs.get(toks[:p + 1], 0) + 1
-            inserted[toks] = inserted.get(toks, 0) + 1
+                holders.setdefault(toks[:p + 1], []).append(owner)
+            inserted[(toks, owner)] = inserted.get((toks, owner), 0) + 1
         elif kind == "release":
+            owner = int(op[2]) if len(op) > 2 else -1
             if n == 0:
                 continue
-            if inserted.get(toks, 0) == 0:
-                raise ValueError("release of a sequence with no insert left to undo")
-            inserted[toks] -= 1
+            if inserted.get((toks, owner), 0) == 0:
+                raise ValueError("release of a sequence with no insert by this owner left to undo")
+            inserted[(toks, owner)] -= 1
             for p in win:
-                key = toks[:p + 1]
-                refs[key] = max(0, refs.get(key, 0) - 1)
+                h = holders.get(toks[:p + 1], [])
+                if owner in h:
+                    h.remove(owner)
         elif kind == "evict":
             lo, hi = op[2], op[3]
             for p in range(max(0, lo), min(n, hi)):
                 if toks[:p + 1] in cached:
-                    refs[toks[:p + 1]] = 0
-        elif kind == "match":
+                    holders[toks[:p + 1]] = []
+        elif kind in ("match", "match_slots"):
             m = 0
             while m < n and toks[:m + 1] in cached:
                 m += 1
             best = 0
             for L in range(0, m + 1):
-                if all(refs.get(toks[:q + 1], 0) > 0 for q in range(max(0, L - window), L)):
+                if all(len(holders.get(toks[:q + 1], [])) > 0 for q in range(max(0, L - window), L)):
                     best = L
-            out.append((m, best))
+            if kind == "match":
+                out.append((m, best))
+            else:
+                slots = [set() for _ in range(window)]
+                for q in range(max(0, best - window), best):
+                    slots[q % window] = set(holders[toks[:q + 1]])
+                out.append((m, best, slots))
         else:
             raise ValueError(kind)
     return out
-

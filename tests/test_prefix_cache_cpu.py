@@ -68,7 +68,7 @@ def test_worked_example():
     assert _replay_library(W, ops) == [(10, 10), (8, 0), (7, 7), (5, 0), (7, 0), (10, 10)]
 
 
-def _random_ops(rng, W, n_ops, alpha):
+def _random_ops(rng, W, n_ops, alpha, owners=False):
     base = [list(rng.integers(0, alpha, size=int(rng.integers(0, 30)))) for _ in range(3)]
     cached = []
     ops = []
@@ -77,22 +77,23 @@ def _random_ops(rng, W, n_ops, alpha):
         if r < 0.3:
             b = base[int(rng.integers(0, 3))]
             seq = b[:int(rng.integers(0, len(b) + 1))] + list(rng.integers(0, alpha, size=int(rng.integers(0, 12))))
-            ops.append(("insert", seq))
-            cached.append(seq)
+            own = int(rng.integers(0, 4)) if owners else -1
+            ops.append(("insert", seq, own))
+            cached.append((seq, own))
         elif r < 0.4 and cached:
-            seq = cached.pop(int(rng.integers(0, len(cached))))
-            ops.append(("release", seq))
+            seq, own = cached.pop(int(rng.integers(0, len(cached))))
+            ops.append(("release", seq, own))
         elif r < 0.55 and cached:
-            seq = cached[int(rng.integers(0, len(cached)))]
+            seq = cached[int(rng.integers(0, len(cached)))][0]
             lo = int(rng.integers(0, len(seq) + 2))
             ops.append(("evict", seq, lo, lo + int(rng.integers(0, 6))))
         else:
             if cached and rng.random() < 0.7:
-                src = cached[int(rng.integers(0, len(cached)))]
+                src = cached[int(rng.integers(0, len(cached)))][0]
                 q = src[:int(rng.integers(0, len(src) + 1))] + list(rng.integers(0, alpha, size=int(rng.integers(0, 4))))
             else:
                 q = list(rng.integers(0, alpha, size=int(rng.integers(0, 20))))
-            ops.append(("match", q))
+            ops.append(("match_slots" if owners else "match", q))
     return ops
 
 
@@ -101,11 +102,13 @@ def _replay_library(W, ops):
     out = []
     for op in ops:
         if op[0] == "insert":
-            t.insert(op[1])
+            t.insert(op[1], *op[2:])
         elif op[0] == "release":
-            t.release(op[1])
+            t.release(op[1], *op[2:])
         elif op[0] == "evict":
             t.evict_swa(op[1], op[2], op[3])
+        elif op[0] == "match_slots":
+            out.append(t.match_slots(op[1]))
         else:
             out.append(t.match(op[1]))
     t.close()
@@ -118,6 +121,38 @@ def test_library_matches_model(W, alpha, seed):
     for _ in range(20):
         ops = _random_ops(rng, W, 60, alpha)
         assert _replay_library(W, ops) == oracle.prefix_cache_replay(W, ops)
+
+
+@pytest.mark.parametrize("W,alpha,seed", [(1, 3, 11), (3, 3, 12), (4, 2, 13), (8, 5, 14)])
+def test_library_slot_owners_match_model(W, alpha, seed):
+    # with owners (ring rows): every slot of the resumed window names one of the model's holders of
+    # the position it keeps, and the other slots are -1
+    rng = np.random.default_rng(seed)
+    for _ in range(20):
+        ops = _random_ops(rng, W, 60, alpha, owners=True)
+        got = _replay_library(W, ops)
+        want = oracle.prefix_cache_replay(W, ops)
+        assert len(got) == len(want)
+        for (m, L, slots), (m2, L2, sets) in zip(got, want):
+            assert (m, L) == (m2, L2)
+            for s in range(W):
+                if sets[s]:
+                    assert int(slots[s]) in sets[s], (s, slots, sets)
+                else:
+                    assert slots[s] == -1
+
+
+def test_owner_released_after_eviction_and_reinsert():
+    # A's window covers position 5; it is evicted, then B (same path) is inserted and holds it
+    # afresh; releasing A must not take B's copy away
+    W = 4
+    A = [1, 2, 3, 4, 5, 6]
+    B = A + [7]
+    ops = [("insert", A, 0), ("evict", A, 5, 6), ("insert", B, 1), ("release", A, 0), ("match_slots", B)]
+    want = oracle.prefix_cache_replay(W, ops)
+    assert want[0][:2] == (7, 7) and want[0][2][5 % W] == {1}
+    got = _replay_library(W, ops)
+    assert got[0][:2] == (7, 7) and list(got[0][2]) == [1, 1, 1, 1]
 
 
 def test_batch_equals_single_and_stats():
@@ -167,6 +202,8 @@ def test_release_needs_an_insert_of_exactly_those_tokens():
     # the rejected releases changed nothing: both windows still count
     assert t.match(A) == (10, 10)
     assert t.match(A[:6]) == (6, 6)
+    with pytest.raises(hs.HswaError):
+        t.release(A[:6], 3)  # inserted by owner -1, not by owner 3
     t.release(A[:6])
     with pytest.raises(hs.HswaError):
         t.release(A[:6])  # its one insert is already undone
