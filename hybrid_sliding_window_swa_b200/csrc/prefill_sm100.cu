@@ -14,10 +14,13 @@
 // prefill_narrow.cu (launch_prefill dispatches). The per-row softmax step and the output
 // epilogue are shared with it (prefill_tile.cuh).
 //
-// Work unit = 2 query tiles of 128 rows (one batch row b, one query head h). The grid
-// is persistent (one CTA per SM) and walks the units in a static round-robin, heaviest
-// (latest query tiles) first; consecutive CTAs take the query heads of one KV group
-// so their K/V tiles are shared through L2.
+// Work unit: two 128-row query tiles that share every key tile. With an even number G of query
+// heads per KV head the two tiles are the same rows of two heads of one GQA group (unit = query
+// tile, batch row, KV head, head pair): they need the same key tiles, so each K/V tile loaded into
+// shared memory feeds both and the two slots' work is equal. With odd G the unit is two
+// consecutive query tiles of one head. The grid is persistent (one CTA per SM) and walks the
+// units in a static round-robin, heaviest (latest query tiles) first; consecutive CTAs take the
+// heads of one KV group so their K/V tiles are shared through L2.
 //   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one thread per
 //               row (TMEM lane); all 128 scores of a row in registers, online max/sum
 //               in the exp2 domain with lazy O rescaling, MUFU exponentials (an FMA-pipe
@@ -66,7 +69,9 @@ struct Params {
   int full_layer;
   int64_t pages;
   float scale_log2;
-  int n_pairs;
+  int n_pairs;     // pairs of query tiles per (batch row, head)   (G odd)
+  int n_tiles;     // query tiles per batch row                    (G even)
+  int head_pairs;  // 1: a unit is one query tile of two heads of a GQA group
   int n_units;
   int64_t max_start;  // largest start position that keeps every position below 2^31
   int* err;
@@ -98,7 +103,8 @@ struct Bars {
 // Geometry of one work unit, computed identically by every role.
 // Positions are below 2^31 (checked on the host against start_pos bounds on the device).
 struct Geo {
-  int b, h, g;
+  int b, g;
+  int hq[NQT];           // query head of each slot
   int P;                 // absolute position of the chunk's first row
   int t[NQT];            // query tile index within the chunk
   bool act[NQT];
@@ -118,12 +124,34 @@ __device__ __forceinline__ int key_base(const Params& p, const Geo& G, int j) {
 }
 
 __device__ __forceinline__ void make_geo(const Params& p, int unit, Geo& G) {
-  const int per_pair = p.B * p.Hq;
-  const int pair = p.n_pairs - 1 - unit / per_pair;  // latest (longest causal) tiles first
-  const int rem = unit % per_pair;
-  G.b = rem / p.Hq;
-  G.h = rem % p.Hq;
-  G.g = G.h / p.G;
+  int tq[NQT];
+  if (p.head_pairs) {
+    const int n_hp = p.G >> 1;
+    const int per_t = p.B * p.Hkv * n_hp;
+    const int t = p.n_tiles - 1 - unit / per_t;  // latest (longest causal) tiles first
+    int rem = unit % per_t;
+    G.b = rem / (p.Hkv * n_hp);
+    rem -= G.b * (p.Hkv * n_hp);
+    G.g = rem / n_hp;
+    const int hp = rem - G.g * n_hp;
+#pragma unroll
+    for (int q = 0; q < NQT; ++q) {
+      tq[q] = t;
+      G.hq[q] = G.g * p.G + 2 * hp + q;
+    }
+  } else {
+    const int per_pair = p.B * p.Hq;
+    const int pair = p.n_pairs - 1 - unit / per_pair;  // latest (longest causal) tiles first
+    const int rem = unit % per_pair;
+    G.b = rem / p.Hq;
+    const int h = rem % p.Hq;
+    G.g = h / p.G;
+#pragma unroll
+    for (int q = 0; q < NQT; ++q) {
+      tq[q] = pair * NQT + q;
+      G.hq[q] = h;
+    }
+  }
   int64_t P = p.start_pos ? p.start_pos[G.b] : 0;
   if (P < 0 || P > p.max_start) {  // positions must stay below 2^31
     record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
@@ -134,7 +162,7 @@ __device__ __forceinline__ void make_geo(const Params& p, int unit, Geo& G) {
   G.je = INT32_MIN;
 #pragma unroll
   for (int q = 0; q < NQT; ++q) {
-    G.t[q] = pair * NQT + q;
+    G.t[q] = tq[q];
     const int r0 = G.t[q] * BM;
     G.act[q] = r0 < p.n_q;
     G.i0[q] = G.i1[q] = G.jlo[q] = 0;
@@ -195,7 +223,7 @@ __device__ void producer(const Params& p, uint8_t* smem, Bars* bars, const CUten
       for (int q = 0; q < NQT; ++q) {
         if (!G.act[q]) continue;
         for (int dh = 0; dh < D / 64; ++dh)
-          tma_load_4d(smem + L::Q_OFF + q * L::TILE + dh * L::BLOCK, tm_q, &bars->q_full, dh * 64, G.h,
+          tma_load_4d(smem + L::Q_OFF + q * L::TILE + dh * L::BLOCK, tm_q, &bars->q_full, dh * 64, G.hq[q],
                       G.t[q] * BM, G.b);
       }
     }
@@ -439,8 +467,8 @@ __device__ void softmax_wg(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
     if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
     ++no;
     tc_fence_after();
-    store_output<D>(trow, o_col, l, smem + L::O_OFF + q * L::BLOCK + wq * 4096, lane, tm_o, G.h, qt * BM + wq * 32,
-                    G.b, p.n_q);
+    store_output<D>(trow, o_col, l, smem + L::O_OFF + q * L::BLOCK + wq * 4096, lane, tm_o, q ? G.hq[1] : G.hq[0],
+                    qt * BM + wq * 32, G.b, p.n_q);
     // O of this query tile has been read: the next unit's first P V may overwrite it
     // (ordered by this warpgroup's next p_full arrival).
     tc_fence_before();
@@ -546,10 +574,13 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
   p.pages = D.pages_per_full_layer;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)Lc.d));
   p.n_pairs = (int)((Lc.n_q + BM * NQT - 1) / (BM * NQT));
+  p.n_tiles = (int)((Lc.n_q + BM - 1) / BM);
+  p.head_pairs = (p.G % 2) == 0 ? 1 : 0;
   p.max_start = 0x7fffffffLL - Lc.n_q - 2 * BN;
   p.err = pool->err;
   if (Lc.n_q == 0 || Lc.B == 0) return HSWA_OK;
-  const int64_t units = (int64_t)p.n_pairs * Lc.B * Lc.Hq;
+  const int64_t units = p.head_pairs ? (int64_t)p.n_tiles * Lc.B * Lc.Hkv * (p.G / 2)
+                                     : (int64_t)p.n_pairs * Lc.B * Lc.Hq;
   if (units > 0x7fffffff) {
     set_error("prefill: too many work units");
     return HSWA_ERR_UNSUPPORTED_SHAPE;

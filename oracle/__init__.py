@@ -53,6 +53,14 @@ def _load():
         L.orc_kv_bytes.argtypes = [i64, i64, i64, i64, i64]
         L.orc_hybrid_kv_ratio.restype = ctypes.c_double
         L.orc_hybrid_kv_ratio.argtypes = [i64, i64, i64, i64]
+        L.orc_attention_kv64.restype = i32
+        L.orc_attention_kv64.argtypes = [p, p, i64, i32, p, p, i64, i64, i32, i32, i64, p, i32]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_double]
+        L.orc_e4m3_quantize.restype = i32
+        L.orc_e4m3_quantize.argtypes = [p, i64, ctypes.c_float, p]
         _lib = L
     return _lib
 
@@ -100,6 +108,55 @@ def attention(q, q_pos, k, v, window: int, key_base: int = 0, n_threads: int | N
     if rc != 0:
         raise ValueError("oracle attention: a needed key position is outside the given keys")
     return out
+
+
+def attention_kv64(q, q_pos, k, v, window: int, key_base: int = 0, n_threads: int | None = None) -> np.ndarray:
+    """``attention`` with float64 keys and values [n_keys, Hkv, d] (dequantized FP8 entries, or a mix
+    of those and bf16 ones); q is bf16 [n_rows, Hq, d]."""
+    qb = _bits(q)
+    k64 = np.ascontiguousarray(np.asarray(k, dtype=np.float64))
+    v64 = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    assert qb.ndim == 3 and k64.ndim == 3 and v64.shape == k64.shape
+    n_rows, hq, d = qb.shape
+    n_keys, hkv, d2 = k64.shape
+    assert d == d2
+    pos = np.ascontiguousarray(np.asarray(q_pos, dtype=np.int64))
+    out = np.empty((n_rows, hq, d), dtype=np.float64)
+    rc = _load().orc_attention_kv64(qb.ctypes.data, pos.ctypes.data, n_rows, hq, k64.ctypes.data, v64.ctypes.data,
+                                    key_base, n_keys, hkv, d, window, out.ctypes.data, n_threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle attention: a needed key position is outside the given keys")
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of FP8 E4M3 codes (uint8 array)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    L = _load()
+    return np.array([L.orc_e4m3_decode(int(x)) for x in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes of float64 values (nearest, ties to even, saturating at +-448)."""
+    a = np.asarray(x, dtype=np.float64)
+    L = _load()
+    return np.array([L.orc_e4m3_encode(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def e4m3_quantize(x, scale: float) -> np.ndarray:
+    """E4M3 codes of bf16 data x (torch bf16 tensor or uint16 bits) stored with scale `scale`:
+    encode(fp32(x) * fp32(1 / scale))."""
+    b = _bits(x)
+    out = np.empty(b.shape, dtype=np.uint8)
+    rc = _load().orc_e4m3_quantize(b.ctypes.data, b.size, float(scale), out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle e4m3_quantize: bad arguments")
+    return out
+
+
+def e4m3_dequantize(codes, scale: float) -> np.ndarray:
+    """The values an FP8 cache holds: decode(code) * scale, in float64 (exact)."""
+    return e4m3_decode(codes) * np.float64(np.float32(scale))
 
 
 def window_safe_len(match_len, cached_len, slot_valid, window: int) -> np.ndarray:

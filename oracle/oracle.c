@@ -45,8 +45,10 @@ typedef struct {
   const int64_t* q_pos;
   int64_t n_rows;
   int n_q_heads;
-  const uint16_t* k;
+  const uint16_t* k;   /* bf16 keys and values, or ... */
   const uint16_t* v;
+  const double* k64;   /* ... fp64 ones (dequantized FP8 cache entries) when these are set */
+  const double* v64;
   int64_t key_base, n_keys;
   int n_kv_heads, head_dim;
   int64_t window;
@@ -54,6 +56,12 @@ typedef struct {
   int64_t first, last; /* (row, head) work items [first, last) */
   int status;
 } attn_job;
+
+/* Element e of key/value row `row` (relative to key_base) of KV head g. */
+static double kv_at(const uint16_t* b16, const double* f64, int64_t row, int n_kv_heads, int g, int d, int e) {
+  const size_t idx = ((size_t)row * n_kv_heads + g) * d + e;
+  return f64 ? f64[idx] : bf16_to_double(b16[idx]);
+}
 
 static void* attn_worker(void* arg) {
   attn_job* J = (attn_job*)arg;
@@ -86,9 +94,8 @@ static void* attn_worker(void* arg) {
     double mx = -INFINITY;
     for (int64_t j = lo; j <= i; ++j) {
       if (!in_window(i, j, J->window)) continue;
-      const uint16_t* krow = J->k + ((size_t)(j - J->key_base) * J->n_kv_heads + g) * d;
       double dot = 0.0;
-      for (int e = 0; e < d; ++e) dot += qd[e] * bf16_to_double(krow[e]);
+      for (int e = 0; e < d; ++e) dot += qd[e] * kv_at(J->k, J->k64, j - J->key_base, J->n_kv_heads, g, d, e);
       s[j - lo] = dot * scale;
       if (s[j - lo] > mx) mx = s[j - lo];
     }
@@ -100,8 +107,7 @@ static void* attn_worker(void* arg) {
     for (int64_t j = lo; j <= i; ++j) {
       const double p = exp(s[j - lo] - mx);
       denom += p;
-      const uint16_t* vrow = J->v + ((size_t)(j - J->key_base) * J->n_kv_heads + g) * d;
-      for (int e = 0; e < d; ++e) o[e] += p * bf16_to_double(vrow[e]);
+      for (int e = 0; e < d; ++e) o[e] += p * kv_at(J->v, J->v64, j - J->key_base, J->n_kv_heads, g, d, e);
     }
     for (int e = 0; e < d; ++e) o[e] /= denom;
   }
@@ -110,9 +116,10 @@ static void* attn_worker(void* arg) {
   return NULL;
 }
 
-int orc_attention(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n_q_heads,
-                  const uint16_t* k, const uint16_t* v, int64_t key_base, int64_t n_keys,
-                  int n_kv_heads, int head_dim, int64_t window, double* out, int n_threads) {
+static int attention_any(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n_q_heads,
+                         const uint16_t* k, const uint16_t* v, const double* k64, const double* v64,
+                         int64_t key_base, int64_t n_keys, int n_kv_heads, int head_dim, int64_t window,
+                         double* out, int n_threads) {
   if (n_rows < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || window < 0) return -1;
   if (n_q_heads % n_kv_heads != 0) return -1;
   if (n_rows == 0) return 0;
@@ -125,7 +132,7 @@ int orc_attention(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n
   for (int t = 0; t < n_threads; ++t) {
     attn_job* J = &jobs[t];
     J->q = q; J->q_pos = q_pos; J->n_rows = n_rows; J->n_q_heads = n_q_heads;
-    J->k = k; J->v = v; J->key_base = key_base; J->n_keys = n_keys;
+    J->k = k; J->v = v; J->k64 = k64; J->v64 = v64; J->key_base = key_base; J->n_keys = n_keys;
     J->n_kv_heads = n_kv_heads; J->head_dim = head_dim; J->window = window; J->out = out;
     J->first = items * t / n_threads;
     J->last = items * (t + 1) / n_threads;
@@ -139,6 +146,66 @@ int orc_attention(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n
   }
   for (int t = 0; t < n_threads; ++t)
     if (jobs[t].status) return -1;
+  return 0;
+}
+
+int orc_attention(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n_q_heads,
+                  const uint16_t* k, const uint16_t* v, int64_t key_base, int64_t n_keys,
+                  int n_kv_heads, int head_dim, int64_t window, double* out, int n_threads) {
+  return attention_any(q, q_pos, n_rows, n_q_heads, k, v, NULL, NULL, key_base, n_keys, n_kv_heads, head_dim,
+                       window, out, n_threads);
+}
+
+int orc_attention_kv64(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n_q_heads,
+                       const double* k, const double* v, int64_t key_base, int64_t n_keys,
+                       int n_kv_heads, int head_dim, int64_t window, double* out, int n_threads) {
+  return attention_any(q, q_pos, n_rows, n_q_heads, NULL, NULL, k, v, key_base, n_keys, n_kv_heads, head_dim,
+                       window, out, n_threads);
+}
+
+/* OCP 8-bit floating point, E4M3: sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+   infinities; S.1111.111 is NaN; exponent field 0 holds the subnormals 0.mmm * 2^-6. */
+double orc_e4m3_decode(uint8_t code) {
+  const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
+/* Nearest E4M3 value, ties to the even mantissa; magnitudes of 448 and above give +-448 (the
+   largest finite value) instead of NaN; NaN gives 0x7F. Zero keeps its sign. */
+uint8_t orc_e4m3_encode(double x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const double a = fabs(x);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2); /* a in [2^(e2-1), 2^e2) */
+  int ee = e2 - 1;
+  if (ee < -6) ee = -6; /* below 2^-6 the spacing stays 2^-9 (subnormals) */
+  const double step = ldexp(1.0, ee - 3);
+  const double n = a / step; /* exact: a scaled by a power of two */
+  double k = floor(n);
+  const double frac = n - k;
+  if (frac > 0.5 || (frac == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;
+  int ki = (int)k; /* 0 .. 16 */
+  if (ki == 0) return sign;
+  if (ee == -6 && ki < 8) return sign | (uint8_t)ki; /* subnormal */
+  if (ki == 16) {
+    ee += 1;
+    ki = 8;
+  }
+  return sign | (uint8_t)(((ee + 7) << 3) | (ki - 8));
+}
+
+int orc_e4m3_quantize(const uint16_t* x, int64_t n, float scale, uint8_t* out) {
+  if (n < 0 || !(scale > 0.0f)) return -1;
+  const float inv = 1.0f / scale; /* fp32 reciprocal, then an fp32 product per element */
+  for (int64_t i = 0; i < n; ++i) {
+    const float v = (float)bf16_to_double(x[i]) * inv;
+    out[i] = orc_e4m3_encode((double)v);
+  }
   return 0;
 }
 

@@ -53,6 +53,22 @@ int orc_attention(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n
                   const uint16_t* k, const uint16_t* v, int64_t key_base, int64_t n_keys,
                   int n_kv_heads, int head_dim, int64_t window, double* out, int n_threads);
 
+/* orc_attention with fp64 keys and values ([n_keys][n_kv_heads][head_dim]), e.g. entries of an
+ * FP8 KV cache dequantized with orc_e4m3_decode times their scale, mixed with bf16 ones. */
+int orc_attention_kv64(const uint16_t* q, const int64_t* q_pos, int64_t n_rows, int n_q_heads,
+                       const double* k, const double* v, int64_t key_base, int64_t n_keys,
+                       int n_kv_heads, int head_dim, int64_t window, double* out, int n_threads);
+
+/* FP8 E4M3 (OCP 8-bit floating point formats specification: 1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, no infinities, S.1111.111 = NaN, largest finite magnitude 448) -- the storage
+ * format of an FP8 KV cache ("MiMo v2.5 inference optimisation", closing section: quantization
+ * cuts the bits per cached entry and stacks with the sliding window's cut in entries).
+ * decode: the value of a code. encode: round to nearest, ties to even, saturating at +-448.
+ * quantize: out[i] = encode(fp32(bf16 x[i]) * (1.0f / scale)) with both operations in fp32. */
+double orc_e4m3_decode(uint8_t code);
+uint8_t orc_e4m3_encode(double x);
+int orc_e4m3_quantize(const uint16_t* x, int64_t n, float scale, uint8_t* out);
+
 /* Window-safe prefix-match length, by definition.
  * For request r: match length m, cached length C, and a W-bit slot-valid mask
  * (valid[r * ((W + 31) / 32) + s / 32] bit s % 32 for ring slot s).
