@@ -473,11 +473,12 @@ class DecodeBatch:
     (K/V of every cached key in every window, plus Q, the new K/V and O)."""
     launches_per_step = 7 * 3  # plan + decode (+ merge on the full layer) per call
 
-    def __init__(self, hs, n=256, seq_offset=0, Hq=64, Hkv=8, d=128, W=128, nq=4, n_swa=6):
+    def __init__(self, hs, n=256, seq_offset=0, Hq=64, Hkv=8, d=128, W=128, nq=4, n_swa=6, fp8=False):
         self.hs = hs
         dev = "cuda"
         self.n, self.Hq, self.Hkv, self.d, self.W, self.nq, self.n_swa = n, Hq, Hkv, d, W, nq, n_swa
-        self.name = f"hybrid_decode_{n}seq_L1K-256K_6swa_1full_Hq64_Hkv8_d128_4tok"
+        self.fp8 = fp8
+        self.name = f"hybrid_decode_{n}seq_L1K-256K_6swa_1full_Hq64_Hkv8_d128_4tok" + ("_fp8kv" if fp8 else "")
         self.base = 200 + seq_offset * 100000
         u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 4, seq_offset), n)
         self.lens = torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
@@ -486,7 +487,15 @@ class DecodeBatch:
         pps = (lens + nq + 63) // 64
         total_pages = int(pps.sum())
         maxp = int(pps.max())
-        self.pool = hs.kv_pool_create(hs.PoolDesc(n_swa, 1, W, Hkv, d, n, total_pages))
+        fmt = hs.HSWA_KV_FP8_E4M3 if fp8 else hs.HSWA_KV_BF16
+        self.pool = hs.kv_pool_create(hs.PoolDesc(n_swa, 1, W, Hkv, d, n, total_pages, kv_format=fmt))
+        if fp8:
+            # per-head scales of amax / 448 for |x| <= 6 (the N(0, 1) entries use the whole E4M3 range)
+            u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 7, seq_offset), 2 * (n_swa + 1) * Hkv)
+            sc = (6.0 / 448.0 * (0.75 + 0.5 * u)).to(torch.float32).view(n_swa + 1, 2, Hkv).numpy()
+            self.scales = sc
+            for layer in range(n_swa + 1):
+                self.pool.set_scales(layer, sc[layer, 0], sc[layer, 1])
         perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 5, seq_offset), total_pages).to(torch.int32)
         pt = torch.zeros(n, maxp, dtype=torch.int32)
         off = 0
@@ -521,8 +530,9 @@ class DecodeBatch:
         self.ws = torch.empty(hs.hybrid_decode_workspace_size(self.pool, n, nq, Hq, self.maxL), dtype=torch.uint8,
                               device=dev)
         self.outs = [torch.empty_like(self.qs[0]) for _ in range(n_swa + 1)]
-        self.kv_full = self.S * Hkv * d * 2 * 2
-        self.kv_swa = n_swa * n * (W - 1) * Hkv * d * 2 * 2
+        e = 1 if fp8 else 2  # bytes per cached K/V element
+        self.kv_full = self.S * Hkv * d * e * 2
+        self.kv_swa = n_swa * n * (W - 1) * Hkv * d * e * 2
         qo = n * nq * (Hq * 2 + Hkv * 2) * d * 2      # Q + O + new K + new V per layer
         self.bytes = self.kv_full + self.kv_swa + (n_swa + 1) * qo
         self.full_bytes_per_launch = self.kv_full + qo
@@ -560,23 +570,33 @@ class DecodeBatch:
 
     def check_sample(self, oracle):
         """All rows of the two shortest sequences and of the longest one (the most splits to merge) on
-        the full layer, and of two sequences on an SWA layer."""
+        the full layer, and of two sequences on an SWA layer. FP8 pools: against the oracle on the
+        dequantized entries (new tokens included: they enter as the cache will hold them)."""
         lens, nq, Hq, Hkv, d, W = self.lens, self.nq, self.Hq, self.Hkv, self.d, self.W
         order = torch.argsort(lens)
         errs = []
+
+        def attend(layer, b, lo, hi, window, key_base, L):
+            k = gen(synth.TAG_K, layer, self.base + b, lo, hi - lo, Hkv, d, 1.0, "cpu")
+            v = gen(synth.TAG_V, layer, self.base + b, lo, hi - lo, Hkv, d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, layer, self.base + b, L, nq, Hq, d, 1.0, "cpu")
+            if not self.fp8:
+                return oracle.attention(q, L + np.arange(nq), k, v, window, key_base=key_base)
+            kd = np.empty(tuple(k.shape), dtype=np.float64)
+            vd = np.empty(tuple(v.shape), dtype=np.float64)
+            for g in range(Hkv):
+                ks, vs = float(self.scales[layer, 0, g]), float(self.scales[layer, 1, g])
+                kd[:, g] = oracle.e4m3_dequantize(oracle.e4m3_quantize(k[:, g].contiguous(), ks), ks)
+                vd[:, g] = oracle.e4m3_dequantize(oracle.e4m3_quantize(v[:, g].contiguous(), vs), vs)
+            return oracle.attention_kv64(q, L + np.arange(nq), kd, vd, window, key_base=key_base)
+
         for b in [int(order[0]), int(order[1]), int(order[-1])]:
             L = int(lens[b])
-            k = gen(synth.TAG_K, self.full_layer, self.base + b, 0, L + nq, Hkv, d, 1.0, "cpu")
-            v = gen(synth.TAG_V, self.full_layer, self.base + b, 0, L + nq, Hkv, d, 1.0, "cpu")
-            q = gen(synth.TAG_Q, self.full_layer, self.base + b, L, nq, Hq, d, 1.0, "cpu")
-            ref = oracle.attention(q, L + np.arange(nq), k, v, 0)
+            ref = attend(self.full_layer, b, 0, L + nq, 0, 0, L)
             errs.append(np.abs(self.outs[self.full_layer][b].float().cpu().double().numpy() - ref).ravel())
         for b in [int(order[-1]), min(7, self.n - 1)]:
             L = int(lens[b])
-            k = gen(synth.TAG_K, 2, self.base + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
-            v = gen(synth.TAG_V, 2, self.base + b, L - W + 1, W - 1 + nq, Hkv, d, 1.0, "cpu")
-            q = gen(synth.TAG_Q, 2, self.base + b, L, nq, Hq, d, 1.0, "cpu")
-            ref = oracle.attention(q, L + np.arange(nq), k, v, W, key_base=L - W + 1)
+            ref = attend(2, b, L - W + 1, L + nq, W, L - W + 1, L)
             errs.append(np.abs(self.outs[2][b].float().cpu().double().numpy() - ref).ravel())
         e = np.concatenate(errs)
         return float(e.max()), float(e.mean())
@@ -689,10 +709,18 @@ def secondary_results(hs, oracle_mod, hbm, bf16):
     return out
 
 
-def decode_results(hs, oracle_mod, hbm):
+def decode_results(hs, oracle_mod, hbm, with_aux=True):
+    res = decode_step_result(hs, oracle_mod, hbm, fp8=False)
+    res += decode_step_result(hs, oracle_mod, hbm, fp8=True)
+    if with_aux:
+        res += aux_results(hs, oracle_mod)
+    return res
+
+
+def decode_step_result(hs, oracle_mod, hbm, fp8):
+    """The hybrid decode step (7 calls) on a bf16 or an FP8 pool, L2 flushed before each step."""
     dev = "cuda"
-    W = 128
-    wl = DecodeBatch(hs)
+    wl = DecodeBatch(hs, fp8=fp8)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(2):
         wl.step()
@@ -715,9 +743,18 @@ def decode_results(hs, oracle_mod, hbm):
             "unit": "GB/s", "value": round(wl.bytes / ms / 1e6, 1), "ms": round(ms, 3),
             "pct_hbm_peak": round(100 * wl.bytes / ms / 1e6 / hbm, 1), "bytes": wl.bytes, "sum_ctx": wl.S,
             "full_layer_ms": round(ms_full, 3), "full_layer_gbs": round(wl.full_bytes_per_launch / ms_full / 1e6, 1),
+            "kv_format": "fp8_e4m3" if fp8 else "bf16",
             "l2": "flushed (256 MiB write) before each step", "max_abs_err": mx, "mean_abs_err": mean}]
     del wl
     torch.cuda.empty_cache()
+    return res
+
+
+def aux_results(hs, oracle_mod):
+    """window_safe_len over 4096 requests and the host prefix-cache match."""
+    dev = "cuda"
+    W = 128
+    res = []
     # window_safe_len over 4096 requests (bit-exact vs oracle)
     nr = 4096
     C = synth.uniform_int(SEED, synth.stream_id(synth.TAG_MISC, 11), nr, 0, 262144)
@@ -869,6 +906,8 @@ def main():
                     choices=["swa_prefill_16k", "long_context_1m", "hybrid_decode", "swa_chunk_131k",
                              "full_chunk_131k"])
     ap.add_argument("--decode-seqs", type=int, default=256, help="sequences in the hybrid_decode batch")
+    ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
+                    help="storage of the hybrid_decode pool's K/V entries")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -904,7 +943,7 @@ def main():
         peak = bf16_sus  # a seconds-long step: the sustained figure
         peak_name = f"{peak_src} bf16 sustained"
     elif args.workload == "hybrid_decode":
-        wl = DecodeBatch(hs, n=args.decode_seqs, seq_offset=rank)
+        wl = DecodeBatch(hs, n=args.decode_seqs, seq_offset=rank, fp8=args.kv_format == "fp8")
         wl.flops = wl.bytes  # the decode metric counts bytes
         dominant_flops = wl.full_bytes_per_launch
         peak = hbm

@@ -25,13 +25,17 @@ HSWA_ERR_CUDA = -4
 HSWA_ERR_TIMEOUT = -5
 HSWA_ERR_DEVICE_BOUNDS = -6
 
+HSWA_KV_BF16 = 0
+HSWA_KV_FP8_E4M3 = 1
+
 EXPORTED = [
     "kv_pool_layout", "kv_pool_create", "kv_pool_destroy", "kv_pool_append",
     "swa_prefill_fwd", "full_prefill_fwd", "hybrid_decode_workspace_size", "hybrid_decode_fwd",
     "window_safe_len", "hswa_pool_check_error", "hswa_last_error", "hybrid_decode_fwd_noalloc",
     "hswa_selftest_wait_timeout", "hswa_tree_create", "hswa_tree_destroy", "hswa_tree_insert",
     "hswa_tree_release", "hswa_tree_evict_swa", "hswa_tree_match", "hswa_tree_match_batch", "hswa_tree_stats",
-    "hswa_tree_match_slots", "kv_pool_gather_ring",
+    "hswa_tree_match_slots", "kv_pool_gather_ring", "kv_pool_set_scales", "hswa_shard_kv_heads",
+    "hswa_shard_sequences",
 ]
 
 # scratch bytes available to hybrid_decode_fwd_noalloc (HSWA_NOALLOC_SCRATCH_BYTES in hswa.h)
@@ -48,7 +52,7 @@ class PoolDescC(ctypes.Structure):
     _fields_ = [
         ("n_swa_layers", ctypes.c_int32), ("n_full_layers", ctypes.c_int32), ("window", ctypes.c_int32),
         ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
-        ("max_seqs", ctypes.c_int32), ("reserved", ctypes.c_int32), ("pages_per_full_layer", ctypes.c_int64),
+        ("max_seqs", ctypes.c_int32), ("kv_format", ctypes.c_int32), ("pages_per_full_layer", ctypes.c_int64),
     ]
 
 
@@ -85,6 +89,10 @@ def load_library(path: str | None = None):
         "hswa_tree_release": [p, p, i64, ctypes.c_int32],
         "hswa_tree_match_slots": [p, p, i64, ctypes.POINTER(i64), ctypes.POINTER(i64), p],
         "kv_pool_gather_ring": [p, i32, ctypes.c_int32, p, p],
+        "kv_pool_set_scales": [p, i32, p, p],
+        "hswa_shard_kv_heads": [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                ctypes.POINTER(ctypes.c_int32)],
+        "hswa_shard_sequences": [p, ctypes.c_int32, ctypes.c_int32, p, p],
         "hswa_tree_evict_swa": [p, p, i64, i64, i64, ctypes.POINTER(i64)],
         "hswa_tree_match": [p, p, i64, ctypes.POINTER(i64), ctypes.POINTER(i64)],
         "hswa_tree_match_batch": [p, p, p, ctypes.c_int32, p, p],
@@ -133,10 +141,15 @@ class PoolDesc:
     max_seqs: int
     pages_per_full_layer: int
     page_size: int = 64
+    kv_format: int = HSWA_KV_BF16
 
     def c(self) -> PoolDescC:
         return PoolDescC(self.n_swa_layers, self.n_full_layers, self.window, self.n_kv_heads, self.head_dim,
-                         self.page_size, self.max_seqs, 0, self.pages_per_full_layer)
+                         self.page_size, self.max_seqs, self.kv_format, self.pages_per_full_layer)
+
+    @property
+    def fp8(self) -> bool:
+        return self.kv_format == HSWA_KV_FP8_E4M3
 
 
 def kv_pool_layout(desc: PoolDesc) -> tuple[int, int, int]:
@@ -159,13 +172,16 @@ class KVPool:
     def _views(self):
         d = self.desc
         _, swa, _full = kv_pool_layout(d)
+        e = 1 if d.fp8 else 2
         ring_half = d.max_seqs * d.n_swa_layers * d.n_kv_heads * d.window * d.head_dim
         page_half = d.n_full_layers * d.pages_per_full_layer * d.n_kv_heads * d.page_size * d.head_dim
         mem = self.memory
-        ring = mem[: 4 * ring_half].view(torch.bfloat16).view(2, d.max_seqs, d.n_swa_layers, d.n_kv_heads,
-                                                               d.window, d.head_dim)
-        pages = mem[swa: swa + 4 * page_half].view(torch.bfloat16).view(
-            2, d.n_full_layers, d.pages_per_full_layer, d.n_kv_heads, d.page_size, d.head_dim)
+        ring = mem[: 2 * e * ring_half]
+        pages = mem[swa: swa + 2 * e * page_half]
+        if not d.fp8:
+            ring, pages = ring.view(torch.bfloat16), pages.view(torch.bfloat16)
+        ring = ring.view(2, d.max_seqs, d.n_swa_layers, d.n_kv_heads, d.window, d.head_dim)
+        pages = pages.view(2, d.n_full_layers, d.pages_per_full_layer, d.n_kv_heads, d.page_size, d.head_dim)
         return ring, pages
 
     @property
@@ -176,13 +192,19 @@ class KVPool:
 
     @property
     def ring(self) -> torch.Tensor:
-        """[2 (K,V)][max_seqs][n_swa_layers][Hkv][W][d] view of the rolling buffers."""
+        """[2 (K,V)][max_seqs][n_swa_layers][Hkv][W][d] view of the rolling buffers (bf16, or uint8
+        E4M3 codes in an FP8 pool)."""
         return self._views()[0]
 
     @property
     def pages(self) -> torch.Tensor:
-        """[2 (K,V)][n_full_layers][pages][Hkv][page_size][d] view of the paged pool."""
+        """[2 (K,V)][n_full_layers][pages][Hkv][page_size][d] view of the paged pool (bf16, or uint8
+        E4M3 codes in an FP8 pool)."""
         return self._views()[1]
+
+    def set_scales(self, layer: int, k_scale, v_scale):
+        """FP8 pools: K and V scales of `layer`, one per KV head (see kv_pool_set_scales)."""
+        kv_pool_set_scales(self, layer, k_scale, v_scale)
 
     def destroy(self):
         if self.handle is not None:
@@ -207,6 +229,17 @@ def kv_pool_create(desc: PoolDesc, memory: torch.Tensor | None = None, device=No
     d = desc.c()
     _check(L.kv_pool_create(ctypes.byref(d), ctypes.c_void_p(memory.data_ptr()), memory.numel(), ctypes.byref(h)))
     return KVPool(desc, memory, h)
+
+
+def kv_pool_set_scales(pool: KVPool, layer: int, k_scale, v_scale):
+    """FP8 pools: K and V scales of `layer` (sequences of n_kv_heads floats > 0; host values)."""
+    import numpy as np
+    ks = np.ascontiguousarray(np.asarray(k_scale, dtype=np.float32).reshape(-1))
+    vs = np.ascontiguousarray(np.asarray(v_scale, dtype=np.float32).reshape(-1))
+    if ks.size != pool.desc.n_kv_heads or vs.size != pool.desc.n_kv_heads:
+        raise ValueError("one K and one V scale per KV head")
+    _check(load_library().kv_pool_set_scales(pool.handle, layer, ks.ctypes.data_as(ctypes.c_void_p),
+                                             vs.ctypes.data_as(ctypes.c_void_p)))
 
 
 def kv_pool_destroy(pool: KVPool):
@@ -329,6 +362,25 @@ def hybrid_decode_fwd_noalloc(pool: KVPool, layer: int, q: torch.Tensor, k_new: 
         _ptr(ctx_len, torch.int64, "ctx_len"), max_ctx_len, _ptr(seq_ids, torch.int32, "seq_ids"),
         _ptr(page_table, torch.int32, "page_table"), pt_stride, hq, _stream(stream)))
     return o
+
+
+def hswa_shard_kv_heads(n_kv_heads: int, n_ranks: int, rank: int) -> tuple[int, int]:
+    """[head_begin, head_end) of the KV heads rank `rank` owns when prefill is split over n_ranks."""
+    b, e = ctypes.c_int32(), ctypes.c_int32()
+    _check(load_library().hswa_shard_kv_heads(n_kv_heads, n_ranks, rank, ctypes.byref(b), ctypes.byref(e)))
+    return b.value, e.value
+
+
+def hswa_shard_sequences(ctx_len, n_ranks: int):
+    """(rank of each sequence, total context per rank) for decode split over n_ranks (numpy arrays)."""
+    import numpy as np
+    lens = np.ascontiguousarray(np.asarray(ctx_len, dtype=np.int64).reshape(-1))
+    ranks = np.zeros(lens.size, dtype=np.int32)
+    loads = np.zeros(n_ranks, dtype=np.int64)
+    _check(load_library().hswa_shard_sequences(lens.ctypes.data_as(ctypes.c_void_p), lens.size, n_ranks,
+                                               ranks.ctypes.data_as(ctypes.c_void_p),
+                                               loads.ctypes.data_as(ctypes.c_void_p)))
+    return ranks, loads
 
 
 def _tokens(tokens):

@@ -303,6 +303,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Two fp32 -> packed E4M3 pair (OCP FP8; round to nearest even, saturating at +-448): lo in the
+// low byte.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // ---------------------------------------------------------------- packed fp32x2 (sm_100)
 
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {

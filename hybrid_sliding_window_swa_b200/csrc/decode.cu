@@ -30,7 +30,8 @@ namespace {
 
 constexpr int DEC_THREADS = 128;
 constexpr int KB = 64;          // keys per block
-constexpr int NST = 3;          // pipeline stages
+constexpr int NST = 3;          // pipeline stages (bf16 blocks)
+constexpr int NST8 = 6;         // pipeline stages (FP8 blocks: half the bytes, the same bytes in flight)
 #ifndef HSWA_DECODE_SPLIT
 #define HSWA_DECODE_SPLIT 8192
 #endif
@@ -95,6 +96,12 @@ struct DecParams {
   int pt_stride;
   const uint16_t* src_k;  // ring or page base of the layer
   const uint16_t* src_v;
+  const uint8_t* src_k8;  // the same, as bytes
+  const uint8_t* src_v8;
+  const float* k_scale;   // FP8 pools: per KV head of this layer: scale and reciprocal of K and V
+  const float* v_scale;
+  const float* inv_k;
+  const float* inv_v;
   int n_swa, ring_layer, max_seqs;
   int full_layer;
   int64_t pages;
@@ -276,31 +283,76 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// byte offset of 16-byte chunk `c` of row `r` in a [rows][D] bf16 tile, XOR-swizzled
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two fp32 -> packed f16x2 (round to nearest even, saturating at +-65504); lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 codes (low byte, high byte of x's low 16 bits) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(x));
+  return r;
+}
+
+// byte offset of 16-byte chunk `c` of row `r` in a [rows][D] bf16 (or f16) tile, XOR-swizzled
 template <int D>
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return (uint32_t)(r * (D * 2) + ((c ^ (r & 7)) << 4));
 }
 
-template <int D, int MT>
+// byte offset of 16-byte chunk `c` of row `r` in a [rows][D] FP8 tile (rows of D bytes), XOR-swizzled
+// so that the 8 rows an ldmatrix reads fall in distinct banks
+template <int D>
+__device__ __forceinline__ uint32_t sw8_off(int r, int c) {
+  if constexpr (D == 128) return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+  else return (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+}
+
+template <int D, int MT, bool FP8>
 struct DecSmem {
   static constexpr int ROWS = 16 * MT;
-  static constexpr int TILE = KB * D * 2;
+  static constexpr int NS = FP8 ? NST8 : NST;      // pipeline stages
+  static constexpr int TILE = KB * D * (FP8 ? 1 : 2);
   static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = K_OFF + NST * TILE;
-  static constexpr int Q_OFF = V_OFF + NST * TILE;
+  static constexpr int V_OFF = K_OFF + NS * TILE;
+  static constexpr int Q_OFF = V_OFF + NS * TILE;  // Q rows, bf16 (or f16 with FP8 blocks)
   static constexpr int MISC_OFF = Q_OFF + ROWS * D * 2;
-  // merge area aliases the K stages (idle while merging)
+  // merge area aliases the K/V stages (idle while merging)
   static constexpr int ACC_OFF = 0;
   static constexpr int BYTES = MISC_OFF + 4 * ROWS * 4 * 2 + ROWS * 4 * 2 + 64;
-  static_assert(ROWS * D * 4 <= NST * TILE, "merge buffer must fit in the K stages");
+  static_assert(4 * ROWS * (D + 8) * 4 <= 2 * NS * TILE, "merge regions must fit in the K/V stages");
 };
 
-template <int D, int MT>
+// FP8 blocks (pools of E4M3 codes): the block copies move half the bytes; S = Q K^T and O += P V
+// run on f16 MMAs (E4M3 -> f16 is exact) with Q and P in f16, fragments built straight from the
+// FP8 bytes in shared memory:
+//  * K: ldmatrix of an 8-key x 16-byte FP8 matrix gives each thread 4 consecutive dims of one key,
+//    i.e. B-fragment k slots (2l, 2l+1, 2l+8, 2l+9) hold dims (4l, 4l+1, 4l+2, 4l+3); Q is staged
+//    with its dims permuted the same way in each 16-dim group, so every dot product is unchanged.
+//  * V: ldmatrix.trans of the same matrix gives each thread two keys x two adjacent dims; its even
+//    and odd dims form the B fragments of two n-tiles ("even" n-tile 2c holds dims 16c + 2j,
+//    "odd" n-tile 2c + 1 dims 16c + 2j + 1), put back in order when O leaves the registers.
+//  * The K scale of the KV head multiplies the softmax scale; the V scale multiplies O. The new
+//    tokens are quantized with the layer's reciprocal scales as they are staged, the values the
+//    cache holds once they are committed.
+template <int D, int MT, bool FP8>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
-  using SM = DecSmem<D, MT>;
+  using SM = DecSmem<D, MT, FP8>;
   constexpr int ROWS = SM::ROWS;
-  constexpr int CH = D / 8;              // 16-byte chunks per row
+  constexpr int NS = SM::NS;
+  constexpr int CH = FP8 ? D / 16 : D / 8;  // 16-byte chunks per K/V row
   extern __shared__ __align__(128) uint8_t smem[];
   float* m_w = reinterpret_cast<float*>(smem + SM::MISC_OFF);   // [4][ROWS]
   float* l_w = m_w + 4 * ROWS;                                  // [4][ROWS]
@@ -353,9 +405,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     const int b = (a + SPLIT < L) ? a + SPLIT : L;
     const int n_cached_blk = (b - a + KB - 1) / KB;
     const int n_blk = n_cached_blk + (last ? 1 : 0);
-    // source rows of this (sequence, KV head)
-    const uint16_t* ring_k = nullptr;
-    const uint16_t* ring_v = nullptr;
+    // source rows of this (sequence, KV head), as bytes
+    constexpr int RB = FP8 ? D : 2 * D;  // bytes per K/V row
+    const uint8_t* ring_k = nullptr;
+    const uint8_t* ring_v = nullptr;
     bool src_ok = true;
     if (p.window > 0) {
       const int seq = p.seq_ids[s];
@@ -364,26 +417,57 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
         src_ok = false;
       } else {
         const int64_t row0 = (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + g) * p.window;
-        ring_k = p.src_k + row0 * D;
-        ring_v = p.src_v + row0 * D;
+        ring_k = p.src_k8 + row0 * RB;
+        ring_v = p.src_v8 + row0 * RB;
       }
     }
     const int32_t* pt_row = p.page_table ? p.page_table + (int64_t)s * p.pt_stride : nullptr;
 
     // ---- stage Q rows (row = t * G + hh) into shared memory, zero rows >= R
-    for (int idx = tid; idx < ROWS * CH; idx += DEC_THREADS) {
-      const int r = idx / CH, ch = idx % CH;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (r < p.R) {
-        const int t = r / p.G, hh = r % p.G;
-        const uint16_t* src = p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
-        val = *reinterpret_cast<const uint4*>(src);
+    if constexpr (FP8) {
+      // f16, dims of each 16-dim group in the order (0,1,4,5,8,9,12,13 | 2,3,6,7,10,11,14,15)
+      for (int idx = tid; idx < ROWS * (D / 16); idx += DEC_THREADS) {
+        const int r = idx / (D / 16), grp = idx % (D / 16);
+        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (r < p.R) {
+          const int t = r / p.G, hh = r % p.G;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + grp * 16);
+          const uint4 x0 = src[0], x1 = src[1];
+          w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
+          w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
+        }
+        // w[i] holds dims 2i (low half) and 2i + 1 (high half) as bf16
+        uint32_t c0[4], c1[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // dims 4j, 4j+1 -> chunk 0 slot j; dims 4j+2, 4j+3 -> chunk 1 slot j
+          c0[j] = pack_f16x2_sat(__uint_as_float(w[2 * j] << 16), __uint_as_float(w[2 * j] & 0xFFFF0000u));
+          c1[j] = pack_f16x2_sat(__uint_as_float(w[2 * j + 1] << 16), __uint_as_float(w[2 * j + 1] & 0xFFFF0000u));
+        }
+        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, 2 * grp)) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, 2 * grp + 1)) =
+            make_uint4(c1[0], c1[1], c1[2], c1[3]);
       }
-      *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, ch)) = val;
+    } else {
+      for (int idx = tid; idx < ROWS * (D / 8); idx += DEC_THREADS) {
+        const int r = idx / (D / 8), ch = idx % (D / 8);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (r < p.R) {
+          const int t = r / p.G, hh = r % p.G;
+          const uint16_t* src = p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
+          val = *reinterpret_cast<const uint4*>(src);
+        }
+        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, ch)) = val;
+      }
     }
 
     // ---- block loader: block kb2 of this item into stage st. Each copy instruction of the CTA
     // moves CP_ROWS whole rows (contiguous in HBM within a page or a ring run).
+    auto kv_off = [](int r, int c) -> uint32_t {
+      if constexpr (FP8) return sw8_off<D>(r, c);
+      else return sw_off<D>(r, c);
+    };
     auto load_block = [&](int kb2, int st) {
       const uint32_t kdst = s_base + SM::K_OFF + st * SM::TILE;
       const uint32_t vdst = s_base + SM::V_OFF + st * SM::TILE;
@@ -398,11 +482,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
             int slot = slot0 + r;
             if (slot >= p.window) slot = (p.window >= KB) ? slot - p.window : slot % p.window;
             const bool ok = src_ok && r < nvalid;
-            const size_t off = ok ? (size_t)slot * D + cp_chunk * 8 : 0;
-            const uint16_t* sk = ok ? ring_k + off : p.src_k;
-            const uint16_t* sv = ok ? ring_v + off : p.src_v;
-            cp_async_16(kdst + sw_off<D>(r, cp_chunk), sk, ok ? 16u : 0u);
-            cp_async_16(vdst + sw_off<D>(r, cp_chunk), sv, ok ? 16u : 0u);
+            const size_t off = ok ? (size_t)slot * RB + cp_chunk * 16 : 0;
+            const uint8_t* sk = ok ? ring_k + off : p.src_k8;
+            const uint8_t* sv = ok ? ring_v + off : p.src_v8;
+            cp_async_16(kdst + kv_off(r, cp_chunk), sk, ok ? 16u : 0u);
+            cp_async_16(vdst + kv_off(r, cp_chunk), sv, ok ? 16u : 0u);
           }
         } else {
           // a block is exactly one 64-token page (splits start at multiples of 64)
@@ -411,16 +495,45 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           bool ok_page = page >= 0 && page < p.pages;
           if (!ok_page && tid == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
           const int64_t prow = ok_page ? (((int64_t)p.full_layer * p.pages + page) * p.Hkv + g) * 64 : 0;
-          const uint16_t* kbase = p.src_k + prow * D;
-          const uint16_t* vbase = p.src_v + prow * D;
+          const uint8_t* kbase = p.src_k8 + prow * RB;
+          const uint8_t* vbase = p.src_v8 + prow * RB;
 #pragma unroll
           for (int rr = 0; rr < KB; rr += CP_ROWS) {
             const int r = rr + cp_row;
             const bool ok = ok_page && r < nvalid;
-            const int off = ok ? r * D + cp_chunk * 8 : 0;
-            cp_async_16(kdst + sw_off<D>(r, cp_chunk), ok ? kbase + off : p.src_k, ok ? 16u : 0u);
-            cp_async_16(vdst + sw_off<D>(r, cp_chunk), ok ? vbase + off : p.src_v, ok ? 16u : 0u);
+            const int off = ok ? r * RB + cp_chunk * 16 : 0;
+            cp_async_16(kdst + kv_off(r, cp_chunk), ok ? kbase + off : p.src_k8, ok ? 16u : 0u);
+            cp_async_16(vdst + kv_off(r, cp_chunk), ok ? vbase + off : p.src_v8, ok ? 16u : 0u);
           }
+        }
+      } else if constexpr (FP8) {
+        // the new tokens, quantized as the cache will hold them: rows 0 .. n_qt-1, zeros after
+        const float ik = p.inv_k[g], iv = p.inv_v[g];
+        auto q16 = [](const uint16_t* src, float inv) -> uint4 {
+          const uint4 x0 = reinterpret_cast<const uint4*>(src)[0], x1 = reinterpret_cast<const uint4*>(src)[1];
+          const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = pack_e4m3x2(__uint_as_float(w[2 * i] << 16) * inv,
+                                            __uint_as_float(w[2 * i] & 0xFFFF0000u) * inv);
+            const uint32_t hi = pack_e4m3x2(__uint_as_float(w[2 * i + 1] << 16) * inv,
+                                            __uint_as_float(w[2 * i + 1] & 0xFFFF0000u) * inv);
+            o[i] = lo | (hi << 16);
+          }
+          return make_uint4(o[0], o[1], o[2], o[3]);
+        };
+#pragma unroll
+        for (int rr = 0; rr < KB; rr += CP_ROWS) {
+          const int r = rr + cp_row;
+          uint4 qk = make_uint4(0, 0, 0, 0), qv = make_uint4(0, 0, 0, 0);
+          if (r < p.n_qt) {
+            const int64_t row = ((int64_t)s * p.n_qt + r) * p.Hkv + g;
+            qk = q16(p.k_new + row * D + cp_chunk * 16, ik);
+            qv = q16(p.v_new + row * D + cp_chunk * 16, iv);
+          }
+          *reinterpret_cast<uint4*>(smem + SM::K_OFF + st * SM::TILE + kv_off(r, cp_chunk)) = qk;
+          *reinterpret_cast<uint4*>(smem + SM::V_OFF + st * SM::TILE + kv_off(r, cp_chunk)) = qv;
         }
       } else {
         // the new tokens: rows 0 .. n_qt-1 of k_new / v_new, zeros after
@@ -431,14 +544,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           const int64_t row = ((int64_t)s * p.n_qt + (ok ? r : 0)) * p.Hkv + g;
           const uint16_t* sk = p.k_new + row * D + cp_chunk * 8;
           const uint16_t* sv = p.v_new + row * D + cp_chunk * 8;
-          cp_async_16(kdst + sw_off<D>(r, cp_chunk), sk, ok ? 16u : 0u);
-          cp_async_16(vdst + sw_off<D>(r, cp_chunk), sv, ok ? 16u : 0u);
+          cp_async_16(kdst + kv_off(r, cp_chunk), sk, ok ? 16u : 0u);
+          cp_async_16(vdst + kv_off(r, cp_chunk), sv, ok ? 16u : 0u);
         }
       }
     };
 
 #pragma unroll
-    for (int st = 0; st < NST - 1; ++st) {
+    for (int st = 0; st < NS - 1; ++st) {
       if (st < n_blk) load_block(st, st);
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
@@ -469,15 +582,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     // largest window start over the real rows: cached keys at or above it need no mask
     const int lo_max = p.window > 0 ? (L + p.n_qt - 1 - p.window + 1 > 0 ? L + p.n_qt - p.window : 0) : 0;
 
+    const float sl2 = FP8 ? p.scale_log2 * p.k_scale[g] : p.scale_log2;
     for (int kb2 = 0; kb2 < n_blk; ++kb2) {
-      asm volatile("cp.async.wait_group %0;" ::"n"(NST - 2) : "memory");
+      asm volatile("cp.async.wait_group %0;" ::"n"(NS - 2) : "memory");
       __syncthreads();  // block kb2 is visible; every warp is done with block kb2 - 1
       {
-        const int nxt = kb2 + NST - 1;
-        if (nxt < n_blk) load_block(nxt, nxt % NST);
+        const int nxt = kb2 + NS - 1;
+        if (nxt < n_blk) load_block(nxt, nxt % NS);
         asm volatile("cp.async.commit_group;" ::: "memory");
       }
-      const int st = kb2 % NST;
+      const int st = kb2 % NS;
       const uint32_t kt = s_base + SM::K_OFF + st * SM::TILE;
       const uint32_t vt = s_base + SM::V_OFF + st * SM::TILE;
       const uint32_t qt = s_base + SM::Q_OFF;
@@ -489,22 +603,50 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) sacc[mt][nt][0] = sacc[mt][nt][1] = sacc[mt][nt][2] = sacc[mt][nt][3] = 0.f;
+      if constexpr (FP8) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t b0, b1, b2, b3;
-        {
-          const int mi = lane >> 3;
-          const int key = key0 + (mi >> 1) * 8 + (lane & 7);
-          ldsm_x4(kt + sw_off<D>(key, kk * 2 + (mi & 1)), b0, b1, b2, b3);
+        for (int kk = 0; kk < D / 16; kk += 2) {
+          // matrices: keys 0-7 / 8-15 of this warp's slice x dims of groups kk and kk + 1
+          uint32_t r0, r1, r2, r3;
+          {
+            const int mi = lane >> 3;
+            const int key = key0 + (mi & 1) * 8 + (lane & 7);
+            ldsm_x4(kt + sw8_off<D>(key, kk + (mi >> 1)), r0, r1, r2, r3);
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t k0 = h ? r2 : r0, k1 = h ? r3 : r1;
+            const uint32_t b00 = e4m3x2_to_f16x2(k0), b01 = e4m3x2_to_f16x2(k0 >> 16);
+            const uint32_t b10 = e4m3x2_to_f16x2(k1), b11 = e4m3x2_to_f16x2(k1 >> 16);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              uint32_t a0, a1, a2, a3;
+              const int mi = lane >> 3;
+              const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
+              ldsm_x4(qt + sw_off<D>(row, (kk + h) * 2 + (mi >> 1)), a0, a1, a2, a3);
+              mma_f16(sacc[mt][0], a0, a1, a2, a3, b00, b01);
+              mma_f16(sacc[mt][1], a0, a1, a2, a3, b10, b11);
+            }
+          }
         }
+      } else {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          uint32_t a0, a1, a2, a3;
-          const int mi = lane >> 3;
-          const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
-          ldsm_x4(qt + sw_off<D>(row, kk * 2 + (mi >> 1)), a0, a1, a2, a3);
-          mma_bf16(sacc[mt][0], a0, a1, a2, a3, b0, b1);
-          mma_bf16(sacc[mt][1], a0, a1, a2, a3, b2, b3);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t b0, b1, b2, b3;
+          {
+            const int mi = lane >> 3;
+            const int key = key0 + (mi >> 1) * 8 + (lane & 7);
+            ldsm_x4(kt + sw_off<D>(key, kk * 2 + (mi & 1)), b0, b1, b2, b3);
+          }
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            const int mi = lane >> 3;
+            const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
+            ldsm_x4(qt + sw_off<D>(row, kk * 2 + (mi >> 1)), a0, a1, a2, a3);
+            mma_bf16(sacc[mt][0], a0, a1, a2, a3, b0, b1);
+            mma_bf16(sacc[mt][1], a0, a1, a2, a3, b2, b3);
+          }
         }
       }
       // mask (edge blocks only) + online softmax in the exp2 domain with lazy rescaling
@@ -531,7 +673,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int j = nt * 8 + e;
-              const float sv = sacc[mt][nt][hf * 2 + e] * p.scale_log2;
+              const float sv = sacc[mt][nt][hf * 2 + e] * sl2;
               v[nt * 2 + e] = (j >= lo_j && j < hi_j) ? sv : -INFINITY;
             }
           float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
@@ -554,21 +696,55 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           for (int x = 0; x < 4; ++x) pv[x] = ex2_approx(v[x] - moff);
           l_r[mt][hf] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
           // A fragment of P (16 rows x 16 keys): a0/a1 = keys 0-7 (rows r, r+8), a2/a3 = keys 8-15
-          pa[mt][hf + 0] = pack_bf16x2(pv[0], pv[1]);
-          pa[mt][hf + 2] = pack_bf16x2(pv[2], pv[3]);
+          if constexpr (FP8) {
+            pa[mt][hf + 0] = pack_f16x2_sat(pv[0], pv[1]);
+            pa[mt][hf + 2] = pack_f16x2_sat(pv[2], pv[3]);
+          } else {
+            pa[mt][hf + 0] = pack_bf16x2(pv[0], pv[1]);
+            pa[mt][hf + 2] = pack_bf16x2(pv[2], pv[3]);
+          }
         }
       }
       // O += P V  (16 keys x D)
+      if constexpr (FP8) {
 #pragma unroll
-      for (int nd2 = 0; nd2 < D / 16; ++nd2) {
-        uint32_t b0, b1, b2, b3;
-        const int mi = lane >> 3;
-        const int key = key0 + (mi & 1) * 8 + (lane & 7);
-        ldsm_x4_t(vt + sw_off<D>(key, nd2 * 2 + (mi >> 1)), b0, b1, b2, b3);
+        for (int c2 = 0; c2 < D / 16; c2 += 2) {
+          // matrices: keys 0-7 / 8-15 of this warp's slice x the 16 dims of groups c2 and c2 + 1;
+          // transposed, each register holds keys (2l, 2l + 1) x dims (2j, 2j + 1), j = lane / 4
+          uint32_t r0, r1, r2, r3;
+          {
+            const int mi = lane >> 3;
+            const int key = key0 + (mi & 1) * 8 + (lane & 7);
+            ldsm_x4_t(vt + sw8_off<D>(key, c2 + (mi >> 1)), r0, r1, r2, r3);
+          }
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          mma_bf16(o_acc[mt][nd2 * 2 + 0], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b0, b1);
-          mma_bf16(o_acc[mt][nd2 * 2 + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b2, b3);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t v0 = h ? r2 : r0, v1 = h ? r3 : r1;
+            // even dims: bytes 0 and 2 (keys 2l, 2l + 1 of dim 2j); odd dims: bytes 1 and 3
+            const uint32_t be0 = e4m3x2_to_f16x2(__byte_perm(v0, 0u, 0x0020u));
+            const uint32_t be1 = e4m3x2_to_f16x2(__byte_perm(v1, 0u, 0x0020u));
+            const uint32_t bo0 = e4m3x2_to_f16x2(__byte_perm(v0, 0u, 0x0031u));
+            const uint32_t bo1 = e4m3x2_to_f16x2(__byte_perm(v1, 0u, 0x0031u));
+            const int grp = c2 + h;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              mma_f16(o_acc[mt][2 * grp + 0], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], be0, be1);
+              mma_f16(o_acc[mt][2 * grp + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], bo0, bo1);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+          uint32_t b0, b1, b2, b3;
+          const int mi = lane >> 3;
+          const int key = key0 + (mi & 1) * 8 + (lane & 7);
+          ldsm_x4_t(vt + sw_off<D>(key, nd2 * 2 + (mi >> 1)), b0, b1, b2, b3);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            mma_bf16(o_acc[mt][nd2 * 2 + 0], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b0, b1);
+            mma_bf16(o_acc[mt][nd2 * 2 + 1], pa[mt][0], pa[mt][1], pa[mt][2], pa[mt][3], b2, b3);
+          }
         }
       }
     }
@@ -593,7 +769,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     // (now idle) K/V stage buffers; the output pass sums the four regions (no shared atomics)
     constexpr int RS = D + 8;  // padded row stride: a warp's float2 stores hit distinct banks
     float* part_w = reinterpret_cast<float*>(smem + SM::ACC_OFF);  // [4][ROWS][RS]
-    static_assert(4 * ROWS * RS * 4 <= 2 * NST * SM::TILE, "merge regions must fit in the K/V stages");
+    static_assert(4 * ROWS * RS * 4 <= 2 * NS * SM::TILE, "merge regions must fit in the K/V stages");
     __syncthreads();
     for (int r = tid; r < ROWS; r += DEC_THREADS) {
       float M = -INFINITY;
@@ -612,11 +788,21 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
         const int r = mt * 16 + (lane >> 2) + hf * 8;
         const float Mo = m_all[r] == -INFINITY ? 0.f : m_all[r];
         const float f = ex2_approx(m_r[mt][hf] - Mo);
-        float* dst = part_w + (warp * ROWS + r) * RS + (lane & 3) * 2;
+        if constexpr (FP8) {
+          // n-tiles 2c (even dims) and 2c + 1 (odd dims) of group c: this thread's dims 16c + 4l .. + 3
+          float* dst = part_w + (warp * ROWS + r) * RS + (lane & 3) * 4;
 #pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd)
-          *reinterpret_cast<float2*>(dst + nd * 8) =
-              make_float2(o_acc[mt][nd][hf * 2 + 0] * f, o_acc[mt][nd][hf * 2 + 1] * f);
+          for (int c = 0; c < D / 16; ++c)
+            *reinterpret_cast<float4*>(dst + c * 16) =
+                make_float4(o_acc[mt][2 * c][hf * 2 + 0] * f, o_acc[mt][2 * c + 1][hf * 2 + 0] * f,
+                            o_acc[mt][2 * c][hf * 2 + 1] * f, o_acc[mt][2 * c + 1][hf * 2 + 1] * f);
+        } else {
+          float* dst = part_w + (warp * ROWS + r) * RS + (lane & 3) * 2;
+#pragma unroll
+          for (int nd = 0; nd < D / 8; ++nd)
+            *reinterpret_cast<float2*>(dst + nd * 8) =
+                make_float2(o_acc[mt][nd][hf * 2 + 0] * f, o_acc[mt][nd][hf * 2 + 1] * f);
+        }
       }
     __syncthreads();
     // element (r, c) of the merged, unnormalised O
@@ -630,11 +816,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       return x;
     };
     __syncthreads();
+    const float vs = FP8 ? p.v_scale[g] : 1.f;  // the V scale of an FP8 pool multiplies O
     if (nsp == 1) {
       // single split: normalise and write bf16 output rows
       for (int idx = tid; idx < p.R * (D / 8); idx += DEC_THREADS) {
         const int r = idx / (D / 8), ch = idx % (D / 8);
-        const float inv = 1.f / l_all[r];
+        const float inv = vs / l_all[r];
         const float4 lo4 = merged4(r, ch * 8), hi4 = merged4(r, ch * 8 + 4);
         uint4 pk;
         pk.x = pack_bf16x2(lo4.x * inv, lo4.y * inv);
@@ -649,7 +836,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       float* part = reinterpret_cast<float*>(p.ws + p.part_off + (size_t)item * p.part_bytes);
       for (int idx = tid; idx < p.R * (D / 4); idx += DEC_THREADS) {
         const int r = idx / (D / 4), c = (idx % (D / 4)) * 4;
-        *reinterpret_cast<float4*>(part + r * D + c) = merged4(r, c);
+        float4 x = merged4(r, c);
+        if constexpr (FP8) {
+          x.x *= vs; x.y *= vs; x.z *= vs; x.w *= vs;
+        }
+        *reinterpret_cast<float4*>(part + r * D + c) = x;
       }
       for (int r = tid; r < p.R; r += DEC_THREADS) {
         part[p.R * D + r] = m_all[r];
@@ -775,16 +966,16 @@ int64_t max_splits(int window, int64_t max_ctx_len) {
   return nsp < 1 ? 1 : nsp;
 }
 
-template <int D, int MT>
+template <int D, int MT, bool FP8>
 int launch_t(DecParams& p, int n_items_max, int sms, size_t merge_smem, cudaStream_t stream) {
-  using SM = DecSmem<D, MT>;
+  using SM = DecSmem<D, MT, FP8>;
   plan_kernel<<<1, 1024, 0, stream>>>(p);
-  cudaFuncSetAttribute(decode_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::BYTES);
+  cudaFuncSetAttribute(decode_kernel<D, MT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::BYTES);
   int per_sm = 2;
   int grid = sms * per_sm;
   if (grid > n_items_max) grid = n_items_max;
   if (grid < 1) grid = 1;
-  decode_kernel<D, MT><<<grid, DEC_THREADS, SM::BYTES, stream>>>(p);
+  decode_kernel<D, MT, FP8><<<grid, DEC_THREADS, SM::BYTES, stream>>>(p);
   if (merge_smem > 0) {
     if (merge_smem > 48 * 1024)
       cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)merge_smem);
@@ -837,6 +1028,15 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
   p.pt_stride = Lc.pt_stride;
   p.src_k = Lc.window > 0 ? pool->ring_k : pool->page_k;
   p.src_v = Lc.window > 0 ? pool->ring_v : pool->page_v;
+  p.src_k8 = Lc.window > 0 ? pool->ring_k8 : pool->page_k8;
+  p.src_v8 = Lc.window > 0 ? pool->ring_v8 : pool->page_v8;
+  if (pool->fp8) {
+    const int n_layers = D.n_swa_layers + D.n_full_layers;
+    p.k_scale = pool->scales + (size_t)(0 * n_layers + Lc.layer) * D.n_kv_heads;
+    p.v_scale = pool->scales + (size_t)(1 * n_layers + Lc.layer) * D.n_kv_heads;
+    p.inv_k = pool->scales + (size_t)(2 * n_layers + Lc.layer) * D.n_kv_heads;
+    p.inv_v = pool->scales + (size_t)(3 * n_layers + Lc.layer) * D.n_kv_heads;
+  }
   p.n_swa = D.n_swa_layers;
   p.ring_layer = Lc.ring_layer;
   p.max_seqs = D.max_seqs;
@@ -857,10 +1057,14 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
   const int nmax = mi > 0x7fffffff ? 0x7fffffff : (int)mi;
   const size_t msm = decode_merge_smem_bytes(p.n_seqs, p.n_qt, p.Hq, p.Hkv, p.window, p.max_ctx_len);
   const int sms = pool->sms;
-  if (Lc.d == 128) {
-    return p.R <= 16 ? launch_t<128, 1>(p, nmax, sms, msm, stream) : launch_t<128, 2>(p, nmax, sms, msm, stream);
+#define HSWA_DEC(DD, MM, F8) launch_t<DD, MM, F8>(p, nmax, sms, msm, stream)
+  if (pool->fp8) {
+    if (Lc.d == 128) return p.R <= 16 ? HSWA_DEC(128, 1, true) : HSWA_DEC(128, 2, true);
+    return p.R <= 16 ? HSWA_DEC(64, 1, true) : HSWA_DEC(64, 2, true);
   }
-  return p.R <= 16 ? launch_t<64, 1>(p, nmax, sms, msm, stream) : launch_t<64, 2>(p, nmax, sms, msm, stream);
+  if (Lc.d == 128) return p.R <= 16 ? HSWA_DEC(128, 1, false) : HSWA_DEC(128, 2, false);
+  return p.R <= 16 ? HSWA_DEC(64, 1, false) : HSWA_DEC(64, 2, false);
+#undef HSWA_DEC
 }
 
 }  // namespace hswa

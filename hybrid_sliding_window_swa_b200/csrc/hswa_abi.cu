@@ -10,6 +10,7 @@
 
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "internal.h"
 
@@ -41,8 +42,21 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+static bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box);
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
+}
+
+bool make_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                  const uint32_t* box) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides_bytes, box);
+}
+
+static bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     set_error("cuTensorMapEncodeTiled is not available from the driver");
@@ -56,7 +70,7 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
     es[i] = 1;
     if (i + 1 < rank) gs[i] = strides_bytes[i];
   }
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -88,8 +102,12 @@ static int check_desc(const hswa_pool_desc* d) {
     return HSWA_ERR_INVALID_ARG;
   }
   if (d->n_swa_layers < 0 || d->n_full_layers < 0 || d->n_kv_heads < 1 || d->max_seqs < 0 ||
-      d->pages_per_full_layer < 0 || d->reserved != 0) {
-    set_error("invalid pool descriptor (negative count, zero KV heads or reserved != 0)");
+      d->pages_per_full_layer < 0) {
+    set_error("invalid pool descriptor (negative count or zero KV heads)");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (d->kv_format != HSWA_KV_BF16 && d->kv_format != HSWA_KV_FP8_E4M3) {
+    set_error("kv_format %d unknown (HSWA_KV_BF16 or HSWA_KV_FP8_E4M3)", d->kv_format);
     return HSWA_ERR_INVALID_ARG;
   }
   if (d->window < 1) {
@@ -118,6 +136,12 @@ static int check_heads(const hswa_pool* pool, int n_q_heads) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// FP8 pools: [4][n_layers][Hkv] float32 scales, rounded up to 256 bytes; 0 for bf16 pools.
+static size_t scale_bytes(const hswa_pool_desc* d) {
+  if (d->kv_format != HSWA_KV_FP8_E4M3) return 0;
+  return round256(4 * sizeof(float) * (size_t)(d->n_swa_layers + d->n_full_layers) * d->n_kv_heads);
+}
+
 }  // namespace hswa
 
 using namespace hswa;
@@ -129,14 +153,16 @@ const char* hswa_last_error(void) { return g_err; }
 int kv_pool_layout(const hswa_pool_desc* desc, size_t* bytes_total, size_t* bytes_swa, size_t* bytes_full) {
   int rc = check_desc(desc);
   if (rc) return rc;
-  const size_t e = 2;
+  const bool fp8 = desc->kv_format == HSWA_KV_FP8_E4M3;
+  const size_t e = fp8 ? 1 : 2;
   const size_t swa = round256(2 * (size_t)desc->max_seqs * desc->n_swa_layers * desc->n_kv_heads *
                               (size_t)desc->window * desc->head_dim * e);
   const size_t full = round256(2 * (size_t)desc->n_full_layers * (size_t)desc->pages_per_full_layer *
                                desc->n_kv_heads * (size_t)desc->page_size * desc->head_dim * e);
+  const size_t sc = scale_bytes(desc);
   if (bytes_swa) *bytes_swa = swa;
   if (bytes_full) *bytes_full = full;
-  if (bytes_total) *bytes_total = swa + full + 256;
+  if (bytes_total) *bytes_total = swa + full + sc + 256;
   return HSWA_OK;
 }
 
@@ -149,6 +175,7 @@ int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa
   size_t total = 0, swa = 0, full = 0;
   int rc = kv_pool_layout(desc, &total, &swa, &full);
   if (rc) return rc;
+  const size_t sc_bytes = scale_bytes(desc);
   if (!dev_mem || (reinterpret_cast<uintptr_t>(dev_mem) & 255u) != 0) {
     set_error("kv_pool_create: device memory must be non-null and 256-byte aligned");
     return HSWA_ERR_INVALID_ARG;
@@ -175,19 +202,27 @@ int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa
   p->base = static_cast<uint8_t*>(dev_mem);
   p->bytes_swa = swa;
   p->bytes_full = full;
+  p->bytes_scales = sc_bytes;
+  p->fp8 = desc->kv_format == HSWA_KV_FP8_E4M3;
+  p->esize = p->fp8 ? 1 : 2;
   const size_t ring_half = (size_t)desc->max_seqs * desc->n_swa_layers * desc->n_kv_heads * (size_t)desc->window *
-                           desc->head_dim;
+                           desc->head_dim * p->esize;  // bytes
   const size_t page_half = (size_t)desc->n_full_layers * (size_t)desc->pages_per_full_layer * desc->n_kv_heads *
-                           (size_t)desc->page_size * desc->head_dim;
-  p->ring_k = reinterpret_cast<uint16_t*>(p->base);
-  p->ring_v = p->ring_k + ring_half;
-  p->page_k = reinterpret_cast<uint16_t*>(p->base + swa);
-  p->page_v = p->page_k + page_half;
-  p->err = reinterpret_cast<int*>(p->base + swa + full);
+                           (size_t)desc->page_size * desc->head_dim * p->esize;
+  p->ring_k8 = p->base;
+  p->ring_v8 = p->base + ring_half;
+  p->page_k8 = p->base + swa;
+  p->page_v8 = p->base + swa + page_half;
+  p->ring_k = reinterpret_cast<uint16_t*>(p->ring_k8);
+  p->ring_v = reinterpret_cast<uint16_t*>(p->ring_v8);
+  p->page_k = reinterpret_cast<uint16_t*>(p->page_k8);
+  p->page_v = reinterpret_cast<uint16_t*>(p->page_v8);
+  p->scales = p->fp8 ? reinterpret_cast<float*>(p->base + swa + full) : nullptr;
+  p->err = reinterpret_cast<int*>(p->base + swa + full + sc_bytes);
   const uint64_t D = desc->head_dim;
   p->ring_tma = false;
   const uint64_t ring_rows = (uint64_t)desc->max_seqs * desc->n_swa_layers * desc->n_kv_heads;
-  if (desc->window % 128 == 0 && ring_rows > 0) {
+  if (!p->fp8 && desc->window % 128 == 0 && ring_rows > 0) {
     const uint64_t dims[3] = {D, (uint64_t)desc->window, ring_rows};
     const uint64_t strides[2] = {D * 2, (uint64_t)desc->window * D * 2};
     const uint32_t box[3] = {64, 128, 1};
@@ -200,12 +235,12 @@ int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa
   }
   p->page_tma = false;
   const uint64_t page_rows = (uint64_t)desc->n_full_layers * desc->pages_per_full_layer * desc->n_kv_heads;
-  if (page_rows > 0) {
-    if (page_rows > 0x7FFFFFFFull) {
-      set_error("kv_pool_create: too many (layer, page, head) rows for 32-bit TMA coordinates");
-      delete p;
-      return HSWA_ERR_UNSUPPORTED_SHAPE;
-    }
+  if (page_rows > 0x7FFFFFFFull) {
+    set_error("kv_pool_create: too many (layer, page, head) rows for 32-bit coordinates");
+    delete p;
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (!p->fp8 && page_rows > 0) {
     const uint64_t dims[3] = {D, (uint64_t)desc->page_size, page_rows};
     const uint64_t strides[2] = {D * 2, (uint64_t)desc->page_size * D * 2};
     const uint32_t box[3] = {64, 64, 1};
@@ -216,13 +251,70 @@ int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa
     }
     p->page_tma = true;
   }
+  p->page_tma8 = false;
+  if (p->fp8 && page_rows > 0 && D == 128) {
+    const uint64_t dims[3] = {D, (uint64_t)desc->page_size, page_rows};
+    const uint64_t strides[2] = {D, (uint64_t)desc->page_size * D};
+    const uint32_t box[3] = {128, 64, 1};
+    if (!make_tmap_u8(&p->tm_page_k8, p->page_k8, 3, dims, strides, box) ||
+        !make_tmap_u8(&p->tm_page_v8, p->page_v8, 3, dims, strides, box)) {
+      delete p;
+      return HSWA_ERR_CUDA;
+    }
+    p->page_tma8 = true;
+  }
   cudaError_t e = cudaMemset(p->err, 0, 256);
+  if (e == cudaSuccess && p->fp8) {
+    // every scale 1 (and so every reciprocal 1)
+    std::vector<float> ones(sc_bytes / sizeof(float), 1.0f);
+    e = cudaMemcpy(p->scales, ones.data(), sc_bytes, cudaMemcpyHostToDevice);
+  }
   if (e != cudaSuccess) {
-    set_error("kv_pool_create: clearing the error word failed: %s", cudaGetErrorString(e));
+    set_error("kv_pool_create: initialising the error word or the scales failed: %s", cudaGetErrorString(e));
     delete p;
     return HSWA_ERR_CUDA;
   }
   *out = p;
+  return HSWA_OK;
+}
+
+int kv_pool_set_scales(hswa_pool* pool, int layer, const float* k_scale, const float* v_scale) {
+  if (!pool || !k_scale || !v_scale) {
+    set_error("kv_pool_set_scales: null argument");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  if (!pool->fp8) {
+    set_error("kv_pool_set_scales: the pool stores bf16 entries; scales apply to FP8 pools");
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const hswa_pool_desc& D = pool->desc;
+  const int n_layers = D.n_swa_layers + D.n_full_layers;
+  if (layer < 0 || layer >= n_layers) {
+    set_error("kv_pool_set_scales: layer %d out of range", layer);
+    return HSWA_ERR_INVALID_ARG;
+  }
+  const int H = D.n_kv_heads;
+  std::vector<float> v4(4 * (size_t)H);
+  for (int g = 0; g < H; ++g) {
+    if (!(k_scale[g] > 0.0f) || !(v_scale[g] > 0.0f) || !isfinite(k_scale[g]) || !isfinite(v_scale[g]) ||
+        !isfinite(1.0f / k_scale[g]) || !isfinite(1.0f / v_scale[g])) {
+      set_error("kv_pool_set_scales: scale of KV head %d must be finite and > 0 with a finite reciprocal", g);
+      return HSWA_ERR_INVALID_ARG;
+    }
+    v4[g] = k_scale[g];
+    v4[H + g] = v_scale[g];
+    v4[2 * H + g] = 1.0f / k_scale[g];
+    v4[3 * H + g] = 1.0f / v_scale[g];
+  }
+  if (int rc = check_device(pool, "kv_pool_set_scales")) return rc;
+  for (int w = 0; w < 4; ++w) {
+    cudaError_t e = cudaMemcpy(pool->scales + ((size_t)w * n_layers + layer) * H, v4.data() + (size_t)w * H,
+                               sizeof(float) * H, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      set_error("kv_pool_set_scales: copy failed: %s", cudaGetErrorString(e));
+      return HSWA_ERR_CUDA;
+    }
+  }
   return HSWA_OK;
 }
 
@@ -332,6 +424,7 @@ int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_b
   L.o = o;
   L.pool = pool;
   L.ring_layer = layer;
+  L.layer = layer;
   if ((rc = build_q_map(&L.tm_q, q, B, n_q, n_q_heads, D.head_dim))) return rc;
   if ((rc = build_q_map(&L.tm_k, k, B, n_q, D.n_kv_heads, D.head_dim))) return rc;
   if ((rc = build_q_map(&L.tm_v, v, B, n_q, D.n_kv_heads, D.head_dim))) return rc;
@@ -354,12 +447,17 @@ int full_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, hswa_bf16* 
   int rc = check_heads(pool, n_q_heads);
   if (rc) return rc;
   if ((rc = check_device(pool, "full_prefill_fwd"))) return rc;
+  if (pool->fp8 && D.head_dim != 128) {
+    set_error("full_prefill_fwd: FP8 pages are read with head_dim 128 only");
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
   if (B < 0 || n_q < 0 || B > 65535) {
     set_error("full_prefill_fwd: bad B or n_q");
     return HSWA_ERR_INVALID_ARG;
   }
   if (B == 0 || n_q == 0) return HSWA_OK;
-  if (!q || !o || !aligned16(q) || !aligned16(o) || !page_table || pt_stride < 1 || !pool->page_tma) {
+  if (!q || !o || !aligned16(q) || !aligned16(o) || !page_table || pt_stride < 1 ||
+      !(pool->fp8 ? pool->page_tma8 : pool->page_tma)) {
     set_error("full_prefill_fwd: missing tensor pointer, page table, or pool pages");
     return HSWA_ERR_INVALID_ARG;
   }
@@ -376,9 +474,10 @@ int full_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, hswa_bf16* 
   L.o = o;
   L.pool = pool;
   L.full_layer = layer - D.n_swa_layers;
+  L.layer = layer;
   if ((rc = build_q_map(&L.tm_q, q, B, n_q, n_q_heads, D.head_dim))) return rc;
-  L.tm_k = pool->tm_page_k;
-  L.tm_v = pool->tm_page_v;
+  L.tm_k = pool->fp8 ? pool->tm_page_k8 : pool->tm_page_k;
+  L.tm_v = pool->fp8 ? pool->tm_page_v8 : pool->tm_page_v;
   if ((rc = build_o_map(&L.tm_o, o, B, n_q, n_q_heads, D.head_dim))) return rc;
   return launch_prefill(L, static_cast<cudaStream_t>(stream));
 }
@@ -448,6 +547,7 @@ int prepare_decode(hswa_pool* pool, const char* who, int layer, const uint16_t* 
   }
   *need = decode_workspace_bytes(n_seqs, n_q_per_seq, n_q_heads, D.n_kv_heads, D.head_dim, window, max_ctx_len);
   L->n_seqs = n_seqs;
+  L->layer = layer;
   L->n_qt = n_q_per_seq;
   L->Hq = n_q_heads;
   L->Hkv = D.n_kv_heads;

@@ -13,16 +13,26 @@ struct hswa_pool {
   int sms;           // its multiprocessor count
   int smem_optin;    // its largest opt-in shared memory per block (bytes)
   uint8_t* base;
-  size_t bytes_swa, bytes_full;
+  size_t bytes_swa, bytes_full, bytes_scales;
+  bool fp8;          // entries are FP8 E4M3 codes (1 byte) instead of bf16 (2 bytes)
+  int esize;         // bytes per element
+  // element arrays (uint16_t for bf16 pools; for FP8 pools the same addresses hold bytes, see *8)
   uint16_t* ring_k;  // [max_seqs][n_swa][Hkv][W][d]
   uint16_t* ring_v;
   uint16_t* page_k;  // [n_full][pages][Hkv][page_size][d]
   uint16_t* page_v;
+  uint8_t* ring_k8;  // the same regions as bytes
+  uint8_t* ring_v8;
+  uint8_t* page_k8;
+  uint8_t* page_v8;
+  float* scales;     // FP8: [4][n_layers][Hkv] = K scale, V scale, 1/K scale, 1/V scale (device)
   int* err;          // device error word
   bool ring_tma;     // W is a multiple of 128: ring tiles can be fetched with one TMA box
   CUtensorMap tm_ring_k, tm_ring_v;
   bool page_tma;
   CUtensorMap tm_page_k, tm_page_v;
+  bool page_tma8;                     // FP8 pools with head_dim 128: pages as byte tiles
+  CUtensorMap tm_page_k8, tm_page_v8; // [page_rows][64][128] bytes, 64-row boxes, 128-byte swizzle
 };
 
 namespace hswa {
@@ -38,6 +48,9 @@ int check_device(const hswa_pool* pool, const char* who);
 // dims/strides: innermost first; strides in bytes for dims 1.. (dim 0 is contiguous).
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box);
+// The same for 1-byte elements (FP8 codes), 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                  const uint32_t* box);
 
 int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* seq_ids,
                   const int64_t* start_pos, int n_tok, const uint16_t* k, const uint16_t* v,
@@ -63,6 +76,7 @@ struct PrefillLaunch {
   const hswa_pool* pool;
   int ring_layer;      // SWA layer index within the ring (SWA)
   int full_layer;      // full layer index within the paged pool (full)
+  int layer;           // pool layer index (selects the FP8 scales)
   // tensor maps built by the ABI layer
   CUtensorMap tm_q, tm_k, tm_v;  // tm_k/tm_v: chunk K/V (SWA) or pages (full)
   CUtensorMap tm_o;              // output, stored 32 rows x 64 columns per TMA box
@@ -74,6 +88,7 @@ int launch_prefill_narrow(const PrefillLaunch& L, cudaStream_t stream);
 
 struct DecodeLaunch {
   int n_seqs, n_qt, Hq, Hkv, d;
+  int layer;   // pool layer index (selects the FP8 scales)
   int window;  // >= 1 SWA (ring), 0 full (pages)
   const uint16_t* q;
   const uint16_t* k_new;

@@ -10,13 +10,16 @@
 namespace hswa {
 
 // One thread moves 16 bytes (8 bf16). Rows are (sequence b, token t, KV head g) of d elements.
-template <int D>
+// FP8 pools: the 8 values are stored as E4M3(fp32(x) * fp32(1 / scale)) in 8 bytes, scale of
+// (layer, g) for K and for V.
+template <int D, bool FP8>
 __global__ void __launch_bounds__(256) append_kernel(
     const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int n_seqs, int n_tok, int Hkv,
     const int64_t* __restrict__ start_pos, const int32_t* __restrict__ seq_ids,
     const int32_t* __restrict__ page_table, int pt_stride,
-    uint16_t* __restrict__ dst_k, uint16_t* __restrict__ dst_v, int is_swa, int W, int n_swa, int layer,
-    int max_seqs, int64_t pages, int page_size, int* err) {
+    uint8_t* __restrict__ dst_k, uint8_t* __restrict__ dst_v, int is_swa, int W, int n_swa, int layer,
+    int max_seqs, int64_t pages, int page_size, const float* __restrict__ inv_k,
+    const float* __restrict__ inv_v, int* err) {
   constexpr int VEC = 8;
   constexpr int PER_ROW = D / VEC;
   const int64_t rows = (int64_t)n_seqs * n_tok * Hkv;
@@ -54,10 +57,27 @@ __global__ void __launch_bounds__(256) append_kernel(
     }
     const uint4* src_k = reinterpret_cast<const uint4*>(k + row * D) + c;
     const uint4* src_v = reinterpret_cast<const uint4*>(v + row * D) + c;
-    uint4* out_k = reinterpret_cast<uint4*>(dst_k + dst_row * D) + c;
-    uint4* out_v = reinterpret_cast<uint4*>(dst_v + dst_row * D) + c;
-    *out_k = __ldg(src_k);
-    *out_v = __ldg(src_v);
+    if constexpr (FP8) {
+      const float ik = inv_k[g], iv = inv_v[g];
+      const uint4 a = __ldg(src_k), b = __ldg(src_v);
+      auto q8 = [](const uint4& x, float inv) {
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float f0 = __uint_as_float(w[2 * h] << 16) * inv, f1 = __uint_as_float(w[2 * h] & 0xFFFF0000u) * inv;
+          const float f2 = __uint_as_float(w[2 * h + 1] << 16) * inv,
+                      f3 = __uint_as_float(w[2 * h + 1] & 0xFFFF0000u) * inv;
+          o[h] = (uint32_t)pack_e4m3x2(f0, f1) | ((uint32_t)pack_e4m3x2(f2, f3) << 16);
+        }
+        return make_uint2(o[0], o[1]);
+      };
+      reinterpret_cast<uint2*>(dst_k + dst_row * D)[c] = q8(a, ik);
+      reinterpret_cast<uint2*>(dst_v + dst_row * D)[c] = q8(b, iv);
+    } else {
+      reinterpret_cast<uint4*>(dst_k + dst_row * D * 2)[c] = __ldg(src_k);
+      reinterpret_cast<uint4*>(dst_v + dst_row * D * 2)[c] = __ldg(src_v);
+    }
   }
 }
 
@@ -71,19 +91,23 @@ int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* s
   const int sms = pool->sms;
   const int64_t want = (total + 255) / 256;
   const int grid = (int)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
-  uint16_t* dk = is_swa ? pool->ring_k : pool->page_k;
-  uint16_t* dv = is_swa ? pool->ring_v : pool->page_v;
+  uint8_t* dk = is_swa ? pool->ring_k8 : pool->page_k8;
+  uint8_t* dv = is_swa ? pool->ring_v8 : pool->page_v8;
   const int l = is_swa ? layer : layer - D.n_swa_layers;
-  if (D.head_dim == 128)
-    append_kernel<128><<<grid, 256, 0, stream>>>(k, v, n_seqs, n_tok, D.n_kv_heads, start_pos, seq_ids,
-                                                  page_table, pt_stride, dk, dv, is_swa, D.window,
-                                                  D.n_swa_layers, l, D.max_seqs, D.pages_per_full_layer,
-                                                  D.page_size, pool->err);
-  else
-    append_kernel<64><<<grid, 256, 0, stream>>>(k, v, n_seqs, n_tok, D.n_kv_heads, start_pos, seq_ids,
-                                                 page_table, pt_stride, dk, dv, is_swa, D.window,
-                                                 D.n_swa_layers, l, D.max_seqs, D.pages_per_full_layer,
-                                                 D.page_size, pool->err);
+  const int n_layers = D.n_swa_layers + D.n_full_layers;
+  const float* inv_k = pool->fp8 ? pool->scales + ((size_t)2 * n_layers + layer) * D.n_kv_heads : nullptr;
+  const float* inv_v = pool->fp8 ? pool->scales + ((size_t)3 * n_layers + layer) * D.n_kv_heads : nullptr;
+#define HSWA_APPEND(DD, F8)                                                                                    \
+  append_kernel<DD, F8><<<grid, 256, 0, stream>>>(k, v, n_seqs, n_tok, D.n_kv_heads, start_pos, seq_ids,     \
+                                                   page_table, pt_stride, dk, dv, is_swa, D.window,          \
+                                                   D.n_swa_layers, l, D.max_seqs, D.pages_per_full_layer,     \
+                                                   D.page_size, inv_k, inv_v, pool->err)
+  if (D.head_dim == 128) {
+    if (pool->fp8) HSWA_APPEND(128, true); else HSWA_APPEND(128, false);
+  } else {
+    if (pool->fp8) HSWA_APPEND(64, true); else HSWA_APPEND(64, false);
+  }
+#undef HSWA_APPEND
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("kv_pool_append: launch failed: %s", cudaGetErrorString(e));
@@ -95,11 +119,11 @@ int launch_append(const hswa_pool* pool, int layer, int n_seqs, const int32_t* s
 // Ring row dst of one sliding-window layer, slot by slot from the rows src[s]: one thread moves 16
 // bytes of K and of V. Every ring keeps position p in slot p mod W, so a slot copied from another
 // row keeps its position.
-template <int D>
-__global__ void __launch_bounds__(256) gather_ring_kernel(uint16_t* __restrict__ ring_k, uint16_t* __restrict__ ring_v,
+template <int ROW_BYTES>
+__global__ void __launch_bounds__(256) gather_ring_kernel(uint8_t* __restrict__ ring_k, uint8_t* __restrict__ ring_v,
                                                           const int32_t* __restrict__ src, int W, int Hkv, int n_swa,
                                                           int layer, int max_seqs, int dst, int* err) {
-  constexpr int PER_ROW = D / 8;
+  constexpr int PER_ROW = ROW_BYTES / 16;
   const int64_t total = (int64_t)W * Hkv * PER_ROW;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -113,8 +137,8 @@ __global__ void __launch_bounds__(256) gather_ring_kernel(uint16_t* __restrict__
       record_error(err, HSWA_ERR_DEVICE_BOUNDS);
       continue;
     }
-    const int64_t from = ((((int64_t)sq * n_swa + layer) * Hkv + g) * W + slot) * D;
-    const int64_t to = ((((int64_t)dst * n_swa + layer) * Hkv + g) * W + slot) * D;
+    const int64_t from = ((((int64_t)sq * n_swa + layer) * Hkv + g) * W + slot) * ROW_BYTES;
+    const int64_t to = ((((int64_t)dst * n_swa + layer) * Hkv + g) * W + slot) * ROW_BYTES;
     reinterpret_cast<uint4*>(ring_k + to)[c] = reinterpret_cast<const uint4*>(ring_k + from)[c];
     reinterpret_cast<uint4*>(ring_v + to)[c] = reinterpret_cast<const uint4*>(ring_v + from)[c];
   }
@@ -122,15 +146,17 @@ __global__ void __launch_bounds__(256) gather_ring_kernel(uint16_t* __restrict__
 
 int launch_gather_ring(const hswa_pool* pool, int layer, int dst, const int32_t* src, cudaStream_t stream) {
   const hswa_pool_desc& D = pool->desc;
-  const int64_t total = (int64_t)D.window * D.n_kv_heads * (D.head_dim / 8);
+  const int row_bytes = D.head_dim * pool->esize;  // 64, 128 or 256
+  const int64_t total = (int64_t)D.window * D.n_kv_heads * (row_bytes / 16);
   const int64_t want = (total + 255) / 256;
   const int grid = (int)(want < (int64_t)pool->sms * 8 ? want : (int64_t)pool->sms * 8);
-  if (D.head_dim == 128)
-    gather_ring_kernel<128><<<grid, 256, 0, stream>>>(pool->ring_k, pool->ring_v, src, D.window, D.n_kv_heads,
-                                                       D.n_swa_layers, layer, D.max_seqs, dst, pool->err);
-  else
-    gather_ring_kernel<64><<<grid, 256, 0, stream>>>(pool->ring_k, pool->ring_v, src, D.window, D.n_kv_heads,
-                                                      D.n_swa_layers, layer, D.max_seqs, dst, pool->err);
+#define HSWA_GATHER(RB)                                                                                    \
+  gather_ring_kernel<RB><<<grid, 256, 0, stream>>>(pool->ring_k8, pool->ring_v8, src, D.window, D.n_kv_heads, \
+                                                    D.n_swa_layers, layer, D.max_seqs, dst, pool->err)
+  if (row_bytes == 256) HSWA_GATHER(256);
+  else if (row_bytes == 128) HSWA_GATHER(128);
+  else HSWA_GATHER(64);
+#undef HSWA_GATHER
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("kv_pool_gather_ring: launch failed: %s", cudaGetErrorString(e));

@@ -45,6 +45,11 @@ struct NParams {
   const int32_t* seq_ids;
   const uint16_t* ring_k;
   const uint16_t* ring_v;
+  const uint8_t* ring_k8;  // FP8 pools: the rings as E4M3 codes, and this layer's per-KV-head scales
+  const uint8_t* ring_v8;
+  const float* k_scale;
+  const float* v_scale;
+  int fp8;
   int ring_layer, n_swa, max_seqs, ring_tma;
   float scale_log2;
   int n_tiles;  // query tiles per batch row
@@ -155,8 +160,13 @@ __device__ void kv_producer(const NParams& p, uint8_t* smem, NBars* bars, const 
         if (!seq_ok && lane == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
         const int held_lo = (G.P - p.window > 0) ? G.P - p.window : 0;
         const int64_t base = ring_row * p.window * D;
-        ring_rows_cpasync<D>(p.ring_k + base, seq_ok, held_lo, G.P, p.window, dk, G.P + BN * j, lane);
-        ring_rows_cpasync<D>(p.ring_v + base, seq_ok, held_lo, G.P, p.window, dv, G.P + BN * j, lane);
+        if (p.fp8) {
+          ring_rows_fp8<D>(p.ring_k8 + base, seq_ok, held_lo, G.P, p.window, p.k_scale[G.g], dk, G.P + BN * j, lane);
+          ring_rows_fp8<D>(p.ring_v8 + base, seq_ok, held_lo, G.P, p.window, p.v_scale[G.g], dv, G.P + BN * j, lane);
+        } else {
+          ring_rows_cpasync<D>(p.ring_k + base, seq_ok, held_lo, G.P, p.window, dk, G.P + BN * j, lane);
+          ring_rows_cpasync<D>(p.ring_v + base, seq_ok, held_lo, G.P, p.window, dv, G.P + BN * j, lane);
+        }
         if (lane == 0) mbar_arrive(&bars->kv_full[jj]);
       }
       __syncwarp();
@@ -417,6 +427,14 @@ int launch_prefill_narrow(const PrefillLaunch& Lc, cudaStream_t stream) {
   p.seq_ids = Lc.seq_ids;
   p.ring_k = pool->ring_k;
   p.ring_v = pool->ring_v;
+  p.ring_k8 = pool->ring_k8;
+  p.ring_v8 = pool->ring_v8;
+  p.fp8 = pool->fp8 ? 1 : 0;
+  if (pool->fp8) {
+    const int n_layers = D.n_swa_layers + D.n_full_layers;
+    p.k_scale = pool->scales + (size_t)(0 * n_layers + Lc.layer) * D.n_kv_heads;
+    p.v_scale = pool->scales + (size_t)(1 * n_layers + Lc.layer) * D.n_kv_heads;
+  }
   p.ring_layer = Lc.ring_layer;
   p.n_swa = D.n_swa_layers;
   p.max_seqs = D.max_seqs;

@@ -65,6 +65,12 @@ struct Params {
   int pt_stride;
   const uint16_t* ring_k;
   const uint16_t* ring_v;
+  const uint8_t* ring_k8;  // FP8 pools: the rings as E4M3 codes, and this layer's per-KV-head scales
+  const uint8_t* ring_v8;
+  const float* k_scale;
+  const float* v_scale;
+  int fp8;
+  int conv;  // FP8 pages (full layer): page tiles are converted to bf16 in shared memory by warps 10-11
   int ring_layer, n_swa, max_seqs, ring_tma;
   int full_layer;
   int64_t pages;
@@ -95,6 +101,7 @@ struct Layout {
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE];
+  uint64_t raw_k[NSTAGE], raw_v[NSTAGE];  // FP8 page tiles landed (before conversion)
   uint64_t s_full[NQT], p_full[NQT], o_full[NQT];
   uint64_t v_fix;  // TMA completion of the page tile that holds the last key (before its tail is zeroed)
   uint32_t tmem_base;
@@ -199,7 +206,78 @@ __device__ __forceinline__ void ring_tile_cpasync(const Params& p, const Geo& G,
   if (!seq_ok && lane == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
   const int64_t row_base = seq_ok ? (((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + G.g) * p.window : 0;
   const int held_lo = (G.P - p.window > 0) ? G.P - p.window : 0;
-  ring_rows_cpasync<D>(ring + row_base * D, seq_ok, held_lo, G.P, p.window, dst, kb, lane);
+  if (p.fp8) {
+    const bool is_v = ring == p.ring_v;
+    ring_rows_fp8<D>((is_v ? p.ring_v8 : p.ring_k8) + row_base * D, seq_ok, held_lo, G.P, p.window,
+                     is_v ? p.v_scale[G.g] : p.k_scale[G.g], dst, kb, lane);
+  } else {
+    ring_rows_cpasync<D>(ring + row_base * D, seq_ok, held_lo, G.P, p.window, dst, kb, lane);
+  }
+}
+
+// FP8 page tiles (full layers of an FP8 pool, head_dim 128): the producer loads a tile's 128 rows x
+// 128 codes by TMA (128-byte swizzle) into the upper half of its bf16 stage buffer, which holds the
+// tile's dims 64..127 afterwards; warps 10 and 11 turn it into bf16 in place, row by row (a thread
+// owns whole rows: a row's codes and its upper bf16 half occupy the same 128 bytes, and the thread
+// reads them before it writes). Values are code value times the KV head's scale, rounded to bf16.
+// Rows past the last key of the unit are written as zeros. Then the buffer is handed to the MMA
+// (k_full / v_full, one arrival per converting thread).
+template <int D>
+__device__ void page_converter(const Params& p, uint8_t* smem, Bars* bars) {
+  using L = Layout<D>;
+  static_assert(D == 128, "FP8 page tiles are converted for head_dim 128");
+  const int ct = threadIdx.x - 10 * 32;  // 0 .. 63
+  int it = 0;
+  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
+    Geo G;
+    make_geo(p, unit, G);
+    int kmax = 0;
+    for (int q = 0; q < NQT; ++q)
+      if (G.act[q] && G.i1[q] > kmax) kmax = G.i1[q];
+    for (int j = G.jb; j <= G.je; ++j, ++it) {
+      const int s = it % NSTAGE;
+      const uint32_t ph = (it / NSTAGE) & 1;
+      const int kb = key_base(p, G, j);
+      for (int kv = 0; kv < 2; ++kv) {
+        if (!mbar_wait(kv ? &bars->raw_v[s] : &bars->raw_k[s], ph, p.err)) return;
+        uint8_t* tile = smem + (kv ? L::V_OFF : L::K_OFF) + s * L::TILE;
+        const float sc = kv ? p.v_scale[G.g] : p.k_scale[G.g];
+#pragma unroll 1
+        for (int rr = 0; rr < 2; ++rr) {
+          const int r = ct + 64 * rr;
+          const bool zero = kb + r > kmax;
+          const int sw = r & 7;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            // codes of dims 64 half .. 64 half + 63: 16-byte chunks 4 half .. 4 half + 3 of row r
+            uint4 x[4];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+              x[c4] = zero ? make_uint4(0, 0, 0, 0)
+                           : *reinterpret_cast<const uint4*>(tile + L::BLOCK + r * 128 + (((4 * half + c4) ^ sw) << 4));
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const uint32_t w[4] = {x[c4].x, x[c4].y, x[c4].z, x[c4].w};
+              uint32_t o[8];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                o[2 * i] = e4m3x2_scaled_bf16x2(w[i], sc);
+                o[2 * i + 1] = e4m3x2_scaled_bf16x2(w[i] >> 16, sc);
+              }
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int ch = 2 * c4 + h;  // bf16 chunk of block `half`
+                *reinterpret_cast<uint4*>(tile + half * L::BLOCK + r * 128 + ((ch ^ sw) << 4)) =
+                    make_uint4(o[4 * h], o[4 * h + 1], o[4 * h + 2], o[4 * h + 3]);
+              }
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(kv ? &bars->v_full[s] : &bars->k_full[s]);
+      }
+    }
+  }
 }
 
 template <int D>
@@ -244,7 +322,29 @@ __device__ void producer(const Params& p, uint8_t* smem, Bars* bars, const CUten
         uint64_t* empty = kv ? &bars->v_empty[s] : &bars->k_empty[s];
         uint8_t* dst = smem + (kv ? L::V_OFF : L::K_OFF) + s * L::TILE;
         if (!mbar_wait(empty, ph ^ 1, p.err)) return;
-        if (p.is_full) {
+        if (p.is_full && p.conv) {
+          // FP8 pages: the codes go to the upper half of the stage buffer; page_converter makes bf16
+          uint64_t* raw = kv ? &bars->raw_v[s] : &bars->raw_k[s];
+          if (lane == 0) {
+            mbar_arrive_expect_tx(raw, BN * D);
+            const CUtensorMap* tm = kv ? tm_v : tm_k;
+            for (int half = 0; half < 2; ++half) {
+              const int pos0 = kb + 64 * half;
+              const int lp = pos0 / 64;
+              int64_t row = -1;  // outside the map: zero fill
+              if (pos0 <= kmax) {
+                int32_t page = -1;
+                if (lp < p.pt_stride) page = p.page_table[(int64_t)G.b * p.pt_stride + lp];
+                if (page < 0 || page >= p.pages) {
+                  record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+                } else {
+                  row = ((int64_t)p.full_layer * p.pages + page) * p.Hkv + G.g;
+                }
+              }
+              tma_load_3d(dst + L::BLOCK + half * 64 * 128, tm, raw, 0, 0, (int)row);
+            }
+          }
+        } else if (p.is_full) {
           // Rows of the last page past the last key hold stale memory; P is 0 there, but
           // 0 * NaN would still poison P V, so that V tile is zeroed past kmax before use.
           const bool fix = kv == 1 && kb <= kmax && kmax < kb + BN - 1 && ((kmax + 1) % 64) != 0;
@@ -493,10 +593,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->k_full[s], p.conv ? 64 : 1);  // converting threads, or the loading thread
+      mbar_init(&bars->v_full[s], p.conv ? 64 : 1);
       mbar_init(&bars->k_empty[s], 1);
       mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->raw_k[s], 1);
+      mbar_init(&bars->raw_v[s], 1);
     }
     for (int q = 0; q < NQT; ++q) {
       mbar_init(&bars->s_full[q], 1);
@@ -533,6 +635,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else if (warp == MMA_WARP) {
       if ((threadIdx.x & 31) == 0) mma_issuer<D>(p, smem, bars, tbase);
       __syncwarp();
+    } else if (p.conv) {
+      if constexpr (D == 128) page_converter<D>(p, smem, bars);
     }
   }
 
@@ -566,6 +670,15 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
   p.pt_stride = Lc.pt_stride;
   p.ring_k = pool->ring_k;
   p.ring_v = pool->ring_v;
+  p.ring_k8 = pool->ring_k8;
+  p.ring_v8 = pool->ring_v8;
+  p.fp8 = pool->fp8 ? 1 : 0;
+  p.conv = (pool->fp8 && Lc.window == 0) ? 1 : 0;
+  if (pool->fp8) {
+    const int n_layers = D.n_swa_layers + D.n_full_layers;
+    p.k_scale = pool->scales + (size_t)(0 * n_layers + Lc.layer) * D.n_kv_heads;
+    p.v_scale = pool->scales + (size_t)(1 * n_layers + Lc.layer) * D.n_kv_heads;
+  }
   p.ring_layer = Lc.ring_layer;
   p.n_swa = D.n_swa_layers;
   p.max_seqs = D.max_seqs;
@@ -591,6 +704,10 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
 
   const CUtensorMap& rk = pool->ring_tma ? pool->tm_ring_k : Lc.tm_k;
   const CUtensorMap& rv = pool->ring_tma ? pool->tm_ring_v : Lc.tm_v;
+  if (p.conv && Lc.d != 128) {
+    set_error("prefill: FP8 pages are read with head_dim 128 only");
+    return HSWA_ERR_UNSUPPORTED_SHAPE;
+  }
   if (Lc.d == 128) {
     const int smem = Layout<128>::BYTES + 1024;
     cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -350,5 +350,63 @@ __device__ __forceinline__ void ring_rows_cpasync(const uint16_t* ring_rows, boo
   __syncwarp();
 }
 
+// Two E4M3 codes (the low 16 bits of x) -> their fp32 values times `scale`, packed to bf16x2
+// (the E4M3 -> f16 step is exact; the product rounds once to fp32 and once to bf16).
+__device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t x, float scale) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(x));
+  float lo, hi;
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+  return pack_bf16x2(lo * scale, hi * scale);
+}
+
+// ring_rows_cpasync for a ring of FP8 E4M3 codes: the held rows are dequantized (code value times
+// `scale`) to bf16 in the tile's swizzled layout; the others are zero. One warp, plain loads
+// (eight 16-byte loads in flight per lane); the caller fences and signals as for the cp.async path.
+template <int D>
+__device__ __forceinline__ void ring_rows_fp8(const uint8_t* ring_rows, bool ok, int held_lo, int held_hi, int W,
+                                              float scale, uint8_t* dst, int kb, int lane) {
+  constexpr int CH8 = D / 16;           // 16-code chunks per row
+  constexpr int TOTAL = BN * CH8;       // chunks per tile
+  constexpr int BATCH = 8;
+  static_assert(TOTAL % (32 * BATCH) == 0, "tile chunks");
+  for (int base = 0; base < TOTAL; base += 32 * BATCH) {
+    uint4 x[BATCH];
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const int idx = base + u * 32 + lane;
+      const int r = idx / CH8, c = idx % CH8;
+      const int pos = kb + r;
+      const bool held = ok && pos >= held_lo && pos < held_hi;
+      x[u] = held ? __ldg(reinterpret_cast<const uint4*>(ring_rows + (int64_t)(pos % W) * D + c * 16))
+                  : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const int idx = base + u * 32 + lane;
+      const int r = idx / CH8, c = idx % CH8;
+      const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+      uint32_t o[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[2 * i] = e4m3x2_scaled_bf16x2(w[i], scale);
+        o[2 * i + 1] = e4m3x2_scaled_bf16x2(w[i] >> 16, scale);
+      }
+      // codes 16c .. 16c + 15 -> bf16 chunks 2c and 2c + 1 of the row
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cc = 2 * c + h;
+        const int blk = cc >> 3, ch = cc & 7;
+        *reinterpret_cast<uint4*>(dst + blk * (BM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
+            make_uint4(o[4 * h], o[4 * h + 1], o[4 * h + 2], o[4 * h + 3]);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+
 }  // namespace
 }  // namespace hswa

@@ -59,6 +59,10 @@ extern "C" {
 #define HSWA_ERR_TIMEOUT (-5)
 #define HSWA_ERR_DEVICE_BOUNDS (-6)
 
+/* Storage format of a pool's K/V entries (hswa_pool_desc.kv_format). */
+#define HSWA_KV_BF16 0     /* bf16, as given */
+#define HSWA_KV_FP8_E4M3 1 /* FP8 E4M3 codes with a scale per (layer, KV head) and K/V, see kv_pool_set_scales */
+
 typedef uint16_t hswa_bf16;
 typedef struct hswa_pool hswa_pool;
 
@@ -76,33 +80,47 @@ typedef struct hswa_pool_desc {
   int32_t head_dim;              /* 64 or 128 */
   int32_t page_size;             /* 64 */
   int32_t max_seqs;              /* number of ring rows (sequence ids 0 .. max_seqs-1) */
-  int32_t reserved;              /* must be 0 */
+  int32_t kv_format;             /* HSWA_KV_BF16 or HSWA_KV_FP8_E4M3 */
   int64_t pages_per_full_layer;  /* >= 0 */
 } hswa_pool_desc;
 
 /* Dual-pool sizing ("MiMo v2.5 inference optimisation", section "KV cache redesign":
  * the SWA pool holds W tokens, O(W); the full pool is sized by length, O(N)).
- * Device memory layout, from the base pointer:
- *   ring  K then V : [2][max_seqs][n_swa_layers][n_kv_heads][W][head_dim] bf16
- *   pages K then V : [2][n_full_layers][pages_per_full_layer][n_kv_heads][page_size][head_dim] bf16
+ * Device memory layout, from the base pointer (e = 2 bytes per element for bf16, 1 for FP8):
+ *   ring  K then V : [2][max_seqs][n_swa_layers][n_kv_heads][W][head_dim] elements
+ *   pages K then V : [2][n_full_layers][pages_per_full_layer][n_kv_heads][page_size][head_dim] elements
+ *   scales (FP8 only): [4][n_swa_layers + n_full_layers][n_kv_heads] float32: K scale, V scale,
+ *                    and their fp32 reciprocals
  *   error word     : 256 bytes (int32 device error code + spare)
  * each region starting on a 256-byte boundary.
- * bytes_swa  = 2 * max_seqs * n_swa_layers * n_kv_heads * W * head_dim * 2, rounded up to 256;
- * bytes_full = 2 * n_full_layers * pages * n_kv_heads * page_size * head_dim * 2, rounded up to 256;
- * bytes_total = bytes_swa + bytes_full + 256.  Any output pointer may be NULL. */
+ * bytes_swa  = 2 * max_seqs * n_swa_layers * n_kv_heads * W * head_dim * e, rounded up to 256;
+ * bytes_full = 2 * n_full_layers * pages * n_kv_heads * page_size * head_dim * e, rounded up to 256;
+ * bytes_total = bytes_swa + bytes_full + (FP8: 16 * layers * n_kv_heads rounded up to 256) + 256.
+ * An FP8 entry holds code = E4M3(fp32(x) * fp32(1 / s)) (nearest, ties to even, saturating at
+ * +-448; OCP 8-bit floating point E4M3) and stands for the value E4M3_value(code) * s, where s is
+ * the scale of its layer, KV head and K or V ("MiMo v2.5 inference optimisation", closing
+ * section: quantization cuts the bits per cached entry and stacks with the window's cut in
+ * entries). Any output pointer may be NULL. */
 HSWA_API int kv_pool_layout(const hswa_pool_desc* desc, size_t* bytes_total, size_t* bytes_swa,
                    size_t* bytes_full);
 
 /* Carve a pool out of caller-owned device memory `dev_mem` of `bytes` bytes
  * (>= bytes_total, 256-byte aligned) on the current CUDA device. The library
  * keeps views and TMA descriptors only; it does not initialise the K/V slots,
- * and clears the error word. The caller frees dev_mem after kv_pool_destroy(). */
+ * sets every FP8 scale to 1 and clears the error word (synchronous copies). The
+ * caller frees dev_mem after kv_pool_destroy(). */
 HSWA_API int kv_pool_create(const hswa_pool_desc* desc, void* dev_mem, size_t bytes, hswa_pool** out);
+
+/* FP8 pools: the scales of layer `layer`, k_scale[g] and v_scale[g] for KV head g (host arrays of
+ * n_kv_heads finite values > 0). Entries appended afterwards are quantized with them and every
+ * read of the layer dequantizes with them, so set them before the layer's first append. The copy
+ * is synchronous; no work on the layer may be in flight. HSWA_ERR_INVALID_ARG for a bf16 pool. */
+HSWA_API int kv_pool_set_scales(hswa_pool* pool, int layer, const float* k_scale, const float* v_scale);
 
 /* Release the host-side handle (not the device memory). NULL is accepted. */
 HSWA_API int kv_pool_destroy(hswa_pool* pool);
 
-/* Commit n_tok new tokens per sequence into layer `layer`.
+/* Commit n_tok new tokens per sequence into layer `layer` (quantized to FP8 in an FP8 pool).
  *  k, v       [n_seqs][n_tok][n_kv_heads][head_dim] bf16, token t of row b sits at
  *             absolute position start_pos[b] + t.
  *  start_pos  device int64[n_seqs], >= 0.
@@ -119,7 +137,8 @@ HSWA_API int kv_pool_append(hswa_pool* pool, int layer, int n_seqs, const int32_
                    const int64_t* start_pos, int n_tok, const hswa_bf16* k, const hswa_bf16* v,
                    const int32_t* page_table, int pt_stride, void* stream);
 
-/* Assemble ring row dst_seq of sliding-window layer `layer` slot by slot: for each slot s with
+/* Assemble ring row dst_seq of sliding-window layer `layer` slot by slot (entries are copied as
+ * stored, bf16 or FP8): for each slot s with
  * src_seq[s] >= 0, the K and V rows of slot s (all KV heads) are copied from ring row src_seq[s];
  * slots with src_seq[s] = -1 or src_seq[s] = dst_seq are left as they are. Since every ring keeps
  * position p in slot p mod W, this moves cached window positions held by other sequences' rings
@@ -268,6 +287,25 @@ HSWA_API int hswa_tree_match_batch(const hswa_prefix_tree* tree, const int32_t* 
 
 /* Cached positions (trie nodes) and how many of them hold sliding-window KV. */
 HSWA_API int hswa_tree_stats(const hswa_prefix_tree* tree, int64_t* n_positions, int64_t* n_swa_held);
+
+/* Multi-GPU partition of the hot path (host code; one process per GPU).
+ * Prefill splits by KV head: query head h reads only KV head h / G ("Sliding Window Attention
+ * (SWA) no riron to jisso", section "Mistral: SWA and GQA"), so the rank that owns KV heads
+ * [head_begin, head_end) and query heads [head_begin * G, head_end * G) keeps that slice of every
+ * pool (a pool created with n_kv_heads = head_end - head_begin) and computes those outputs with
+ * no exchange. hswa_shard_kv_heads gives rank `rank` of n_ranks its contiguous, equal range;
+ * HSWA_ERR_UNSUPPORTED_SHAPE unless n_kv_heads is a multiple of n_ranks. */
+HSWA_API int hswa_shard_kv_heads(int32_t n_kv_heads, int32_t n_ranks, int32_t rank, int32_t* head_begin,
+                                 int32_t* head_end);
+
+/* Decode splits by sequence: every sequence, with its ring rows and pages, lives on one rank.
+ * Sequences are taken longest length bucket first (>= 256K, 64K..256K, < 64K tokens; "MiMo v2.5
+ * inference optimisation", section "KV cache redesign"), longest first inside a bucket, and each
+ * goes to the rank with the least total context so far (lowest rank on ties).
+ * ctx_len[n_seqs] (host, >= 0) -> rank_of_seq[n_seqs] (host) and, when not NULL,
+ * load_per_rank[n_ranks] = total context per rank. */
+HSWA_API int hswa_shard_sequences(const int64_t* ctx_len, int32_t n_seqs, int32_t n_ranks, int32_t* rank_of_seq,
+                                  int64_t* load_per_rank);
 
 /* Diagnostic: run, on `stream`, one wait on a barrier that nothing arrives at, through the same
  * bounded wait every kernel uses, with a limit of limit_ns (1 ms .. 2 s; the kernels themselves

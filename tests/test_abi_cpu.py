@@ -54,6 +54,20 @@ def test_layout_matches_kv_bytes_formula(lib):
         assert total == swa + full + 256
 
 
+def test_fp8_layout_halves_the_entries_and_adds_the_scales(lib):
+    # FP8 E4M3 entries take one byte: the KV-bytes formula with 1-byte elements, plus
+    # [4][layers][Hkv] float32 scales
+    for args in [(60, 10, 128, 8, 128, 1, (1 << 20) // 64), (6, 1, 128, 8, 128, 256, 200_000), (1, 1, 1, 1, 64, 3, 7)]:
+        total, swa, full = hs.kv_pool_layout(hs.PoolDesc(*args, kv_format=hs.HSWA_KV_FP8_E4M3))
+        o_swa, o_full = oracle.pool_bytes(*args[:5], 64, args[5], args[6], elem_bytes=1)
+        assert swa == (o_swa + 255) // 256 * 256 and full == (o_full + 255) // 256 * 256
+        scales = (4 * 4 * (args[0] + args[1]) * args[3] + 255) // 256 * 256
+        assert total == swa + full + scales + 256
+    with pytest.raises(hs.HswaError) as e:
+        hs.kv_pool_layout(hs.PoolDesc(1, 1, 128, 8, 128, 1, 4, kv_format=7))
+    assert e.value.code == hs.HSWA_ERR_INVALID_ARG
+
+
 def test_config5_footprint_is_60W_plus_10N_slots(lib):
     n = 1 << 20
     _, swa, full = hs.kv_pool_layout(hs.PoolDesc(60, 10, 128, 8, 128, 1, n // 64))
