@@ -138,6 +138,16 @@ def weak_scaling_value(units_per_rank: float, ws: int, ms_max: float, scale: flo
     return units_per_rank * ws / ms_max / scale
 
 
+def sum_over_ranks(x: float, ws: int) -> float:
+    """Units of work of all ranks together (each rank counts its own)."""
+    if ws == 1:
+        return x
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
 def barrier(ws):
     if ws > 1:
         torch.distributed.barrier()
@@ -154,29 +164,47 @@ class SwaPrefill16k:
     name = "swa_prefill_16k_B2_W4096_Hq32_Hkv8_d128"
 
     @staticmethod
-    def config(ws, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128):
+    def config(ws, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128, shard="replicas", gather_o=False):
         """The config dict of this workload's JSON line (the same for both arms)."""
+        if shard == "heads":
+            par = (f"KV heads split over {ws} ranks ({Hkv // ws} KV / {Hq // ws} query heads each)" +
+                   (", O all-gathered (NCCL) every step" if gather_o else ", O left head-sharded"))
+        else:
+            par = f"independent batches x{ws}"
         return {"workload": SwaPrefill16k.name, "B_per_gpu": B, "seq_len": N, "window": W, "Hq": Hq,
-                "Hkv": Hkv, "head_dim": d, "parallelism": f"independent batches x{ws}",
+                "Hkv": Hkv, "head_dim": d, "parallelism": par,
                 "step": "swa_prefill_fwd + kv_pool_append(ring commit)",
                 "l2": "inputs larger than L2 (Q 268 MB + K/V 134 MB + O 268 MB per step)"}
 
-    def __init__(self, hs, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128, seq_offset=0):
+    def __init__(self, hs, B=2, N=16384, W=4096, Hq=32, Hkv=8, d=128, seq_offset=0, heads=None, gather_o=False):
+        """heads = (g0, g1): this rank's KV heads when the problem is split by KV head (its query
+        heads are [g0 G, g1 G)); the data of a head are those of the unsplit problem."""
         self.hs = hs
         self.B, self.N, self.W, self.Hq, self.Hkv, self.d = B, N, W, Hq, Hkv, d
         self.sigma = 2 ** -0.5
         self.seq_offset = seq_offset
+        G = Hq // Hkv
+        self.g0, self.g1 = heads if heads is not None else (0, Hkv)
+        self.hkv_l, self.hq_l = self.g1 - self.g0, (self.g1 - self.g0) * G
+        h0, h1 = self.g0 * G, self.g1 * G
         dev = "cuda"
-        self.q = torch.stack([gen(synth.TAG_Q, 0, seq_offset + b, 0, N, Hq, d, self.sigma, dev) for b in range(B)])
-        self.k = torch.stack([gen(synth.TAG_K, 0, seq_offset + b, 0, N, Hkv, d, self.sigma, dev) for b in range(B)])
-        self.v = torch.stack([gen(synth.TAG_V, 0, seq_offset + b, 0, N, Hkv, d, self.sigma, dev) for b in range(B)])
+        self.q = torch.stack([gen(synth.TAG_Q, 0, seq_offset + b, 0, N, Hq, d, self.sigma, dev)[:, h0:h1]
+                              for b in range(B)]).contiguous()
+        self.k = torch.stack([gen(synth.TAG_K, 0, seq_offset + b, 0, N, Hkv, d, self.sigma, dev)[:, self.g0:self.g1]
+                              for b in range(B)]).contiguous()
+        self.v = torch.stack([gen(synth.TAG_V, 0, seq_offset + b, 0, N, Hkv, d, self.sigma, dev)[:, self.g0:self.g1]
+                              for b in range(B)]).contiguous()
         self.o = torch.empty_like(self.q)
-        self.pool = hs.kv_pool_create(hs.PoolDesc(1, 0, W, Hkv, d, B, 0))
+        self.pool = hs.kv_pool_create(hs.PoolDesc(1, 0, W, self.hkv_l, d, B, 0))
         self.start = torch.zeros(B, dtype=torch.int64, device=dev)
         self.seq_ids = torch.arange(B, dtype=torch.int32, device=dev)
         pairs = W * (W + 1) // 2 + (N - W) * W if N >= W else N * (N + 1) // 2
-        self.flops = 4 * d * pairs * Hq * B
+        self.flops = 4 * d * pairs * self.hq_l * B  # this rank's share (the whole problem unless split)
         self.tail = min(N, W)
+        self.gather_o = gather_o and torch.distributed.is_initialized()
+        if self.gather_o:
+            ws = torch.distributed.get_world_size()
+            self.o_all = torch.empty((ws,) + tuple(self.o.shape), dtype=self.o.dtype, device=dev)
 
     def step(self, ev=None):
         hs = self.hs
@@ -188,6 +216,9 @@ class SwaPrefill16k:
             ev[-1][1].record()
         # commit the chunk into the rolling buffer (only its last W tokens land)
         hs.kv_pool_append(self.pool, 0, self.k, self.v, self.start, seq_ids=self.seq_ids)
+        if self.gather_o:
+            # every rank gets every head's output: rank-major slices [rank][B][N][Hq / ranks][d]
+            torch.distributed.all_gather_into_tensor(self.o_all, self.o)
 
     launches_per_step = 2
 
@@ -217,6 +248,8 @@ class SwaPrefill16k:
             qr = torch.stack([gen(synth.TAG_Q, 0, self.seq_offset + b, r, 1, self.Hq, self.d, self.sigma, "cpu")[0]
                               for r in rows])
             ref = oracle.attention(qr, np.array(rows), k, v, self.W, key_base=lo)
+            G = self.Hq // self.Hkv
+            ref = ref[:, self.g0 * G:self.g1 * G]  # this rank's heads
             got = self.o[b, list(rows)].float().cpu().double().numpy()
             errs.append(np.abs(got - ref))
         e = np.concatenate([x.ravel() for x in errs])
@@ -473,15 +506,27 @@ class DecodeBatch:
     (K/V of every cached key in every window, plus Q, the new K/V and O)."""
     launches_per_step = 7 * 3  # plan + decode (+ merge on the full layer) per call
 
-    def __init__(self, hs, n=256, seq_offset=0, Hq=64, Hkv=8, d=128, W=128, nq=4, n_swa=6, fp8=False):
+    @staticmethod
+    def batch_lens(n=256, seq_offset=0):
+        """Context lengths of the batch: log-uniform in [1K, 256K] from the seed."""
+        u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 4, seq_offset), n)
+        return torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
+
+    def __init__(self, hs, n=256, seq_offset=0, Hq=64, Hkv=8, d=128, W=128, nq=4, n_swa=6, fp8=False, select=None):
+        """select: indices of the batch's sequences this rank holds when decode is split by sequence
+        (None: all of them); a sequence's data are those of the unsplit batch."""
         self.hs = hs
         dev = "cuda"
-        self.n, self.Hq, self.Hkv, self.d, self.W, self.nq, self.n_swa = n, Hq, Hkv, d, W, nq, n_swa
+        self.Hq, self.Hkv, self.d, self.W, self.nq, self.n_swa = Hq, Hkv, d, W, nq, n_swa
         self.fp8 = fp8
         self.name = f"hybrid_decode_{n}seq_L1K-256K_6swa_1full_Hq64_Hkv8_d128_4tok" + ("_fp8kv" if fp8 else "")
+        all_lens = self.batch_lens(n, seq_offset)
+        self.total_ctx = int(all_lens.sum())
+        self.gidx = list(range(n)) if select is None else [int(i) for i in select]
+        n = len(self.gidx)
+        self.n = n
         self.base = 200 + seq_offset * 100000
-        u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 4, seq_offset), n)
-        self.lens = torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
+        self.lens = all_lens[self.gidx]
         lens = self.lens
         self.S = int(lens.sum())
         pps = (lens + nq + 63) // 64
@@ -507,26 +552,27 @@ class DecodeBatch:
         self.full_layer = n_swa
         for b in range(n):
             L = int(lens[b])
+            sq = self.base + self.gidx[b]  # the sequence's data stream (its index in the whole batch)
             for c0 in range(0, L, 65536):
                 m = min(65536, L - c0)
-                k = gen(synth.TAG_K, self.full_layer, self.base + b, c0, m, Hkv, d, 1.0, dev)[None]
-                v = gen(synth.TAG_V, self.full_layer, self.base + b, c0, m, Hkv, d, 1.0, dev)[None]
+                k = gen(synth.TAG_K, self.full_layer, sq, c0, m, Hkv, d, 1.0, dev)[None]
+                v = gen(synth.TAG_V, self.full_layer, sq, c0, m, Hkv, d, 1.0, dev)[None]
                 hs.kv_pool_append(self.pool, self.full_layer, k, v, torch.tensor([c0], device=dev),
                                   page_table=self.pt[b:b + 1])
             for layer in range(n_swa):
-                k = gen(synth.TAG_K, layer, self.base + b, L - W, W, Hkv, d, 1.0, dev)[None]
-                v = gen(synth.TAG_V, layer, self.base + b, L - W, W, Hkv, d, 1.0, dev)[None]
+                k = gen(synth.TAG_K, layer, sq, L - W, W, Hkv, d, 1.0, dev)[None]
+                v = gen(synth.TAG_V, layer, sq, L - W, W, Hkv, d, 1.0, dev)[None]
                 hs.kv_pool_append(self.pool, layer, k, v, torch.tensor([L - W], device=dev), seq_ids=self.sid[b:b + 1])
         self.ctx = lens.to(dev)
         self.maxL = int(lens.max())
         self.qs, self.kn, self.vn = [], [], []
         for layer in range(n_swa + 1):
-            self.qs.append(torch.stack([gen(synth.TAG_Q, layer, self.base + b, int(lens[b]), nq, Hq, d, 1.0, dev)
-                                        for b in range(n)]))
-            self.kn.append(torch.stack([gen(synth.TAG_K, layer, self.base + b, int(lens[b]), nq, Hkv, d, 1.0, dev)
-                                        for b in range(n)]))
-            self.vn.append(torch.stack([gen(synth.TAG_V, layer, self.base + b, int(lens[b]), nq, Hkv, d, 1.0, dev)
-                                        for b in range(n)]))
+            self.qs.append(torch.stack([gen(synth.TAG_Q, layer, self.base + self.gidx[b], int(lens[b]), nq, Hq, d,
+                                            1.0, dev) for b in range(n)]))
+            self.kn.append(torch.stack([gen(synth.TAG_K, layer, self.base + self.gidx[b], int(lens[b]), nq, Hkv, d,
+                                            1.0, dev) for b in range(n)]))
+            self.vn.append(torch.stack([gen(synth.TAG_V, layer, self.base + self.gidx[b], int(lens[b]), nq, Hkv, d,
+                                            1.0, dev) for b in range(n)]))
         self.ws = torch.empty(hs.hybrid_decode_workspace_size(self.pool, n, nq, Hq, self.maxL), dtype=torch.uint8,
                               device=dev)
         self.outs = [torch.empty_like(self.qs[0]) for _ in range(n_swa + 1)]
@@ -577,9 +623,10 @@ class DecodeBatch:
         errs = []
 
         def attend(layer, b, lo, hi, window, key_base, L):
-            k = gen(synth.TAG_K, layer, self.base + b, lo, hi - lo, Hkv, d, 1.0, "cpu")
-            v = gen(synth.TAG_V, layer, self.base + b, lo, hi - lo, Hkv, d, 1.0, "cpu")
-            q = gen(synth.TAG_Q, layer, self.base + b, L, nq, Hq, d, 1.0, "cpu")
+            sq = self.base + self.gidx[b]
+            k = gen(synth.TAG_K, layer, sq, lo, hi - lo, Hkv, d, 1.0, "cpu")
+            v = gen(synth.TAG_V, layer, sq, lo, hi - lo, Hkv, d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, layer, sq, L, nq, Hq, d, 1.0, "cpu")
             if not self.fp8:
                 return oracle.attention(q, L + np.arange(nq), k, v, window, key_base=key_base)
             kd = np.empty(tuple(k.shape), dtype=np.float64)
@@ -594,7 +641,7 @@ class DecodeBatch:
             L = int(lens[b])
             ref = attend(self.full_layer, b, 0, L + nq, 0, 0, L)
             errs.append(np.abs(self.outs[self.full_layer][b].float().cpu().double().numpy() - ref).ravel())
-        for b in [int(order[-1]), min(7, self.n - 1)]:
+        for b in sorted({int(order[-1]), min(7, self.n - 1)}):
             L = int(lens[b])
             ref = attend(2, b, L - W + 1, L + nq, W, L - W + 1, L)
             errs.append(np.abs(self.outs[2][b].float().cpu().double().numpy() - ref).ravel())
@@ -610,9 +657,10 @@ class DecodeBatch:
             if dt >= budget_s:
                 break
             L = int(self.lens[b])
-            k = gen(synth.TAG_K, self.full_layer, self.base + b, 0, L + self.nq, self.Hkv, self.d, 1.0, "cpu")
-            v = gen(synth.TAG_V, self.full_layer, self.base + b, 0, L + self.nq, self.Hkv, self.d, 1.0, "cpu")
-            q = gen(synth.TAG_Q, self.full_layer, self.base + b, L, self.nq, self.Hq, self.d, 1.0, "cpu")
+            sq = self.base + self.gidx[b]
+            k = gen(synth.TAG_K, self.full_layer, sq, 0, L + self.nq, self.Hkv, self.d, 1.0, "cpu")
+            v = gen(synth.TAG_V, self.full_layer, sq, 0, L + self.nq, self.Hkv, self.d, 1.0, "cpu")
+            q = gen(synth.TAG_Q, self.full_layer, sq, L, self.nq, self.Hq, self.d, 1.0, "cpu")
             t0 = time.perf_counter()
             oracle.attention(q, L + np.arange(self.nq), k, v, 0, n_threads=threads)
             dt += time.perf_counter() - t0
@@ -908,6 +956,10 @@ def main():
     ap.add_argument("--decode-seqs", type=int, default=256, help="sequences in the hybrid_decode batch")
     ap.add_argument("--kv-format", default="bf16", choices=["bf16", "fp8"],
                     help="storage of the hybrid_decode pool's K/V entries")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads", "seqs"],
+                    help="with several GPUs: replicas = every rank its own problem (weak scaling); heads = the "
+                         "16K chunk split by KV head; seqs = the decode batch split by sequence (strong scaling)")
+    ap.add_argument("--gather-o", action="store_true", help="--shard heads: all-gather O over NCCL every step")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -928,6 +980,10 @@ def main():
     torch.cuda.set_device(local)
     import hybrid_sliding_window_swa_b200 as hs
     hs.load_library()
+    if args.shard == "heads" and args.workload != "swa_prefill_16k":
+        raise SystemExit("--shard heads applies to the swa_prefill_16k workload")
+    if args.shard == "seqs" and args.workload != "hybrid_decode":
+        raise SystemExit("--shard seqs applies to the hybrid_decode workload")
     hbm, bf16, bf16_sus, peak_src = peaks()
     decode = args.workload in ("hybrid_decode", "swa_chunk_131k")  # bandwidth-bound: GB/s
     if args.workload in ("swa_chunk_131k", "full_chunk_131k"):
@@ -943,11 +999,21 @@ def main():
         peak = bf16_sus  # a seconds-long step: the sustained figure
         peak_name = f"{peak_src} bf16 sustained"
     elif args.workload == "hybrid_decode":
-        wl = DecodeBatch(hs, n=args.decode_seqs, seq_offset=rank, fp8=args.kv_format == "fp8")
+        if args.shard == "seqs":
+            ranks, _ = hs.hswa_shard_sequences(DecodeBatch.batch_lens(args.decode_seqs).numpy(), ws)
+            wl = DecodeBatch(hs, n=args.decode_seqs, fp8=args.kv_format == "fp8",
+                             select=np.nonzero(ranks == rank)[0])
+        else:
+            wl = DecodeBatch(hs, n=args.decode_seqs, seq_offset=rank, fp8=args.kv_format == "fp8")
         wl.flops = wl.bytes  # the decode metric counts bytes
         dominant_flops = wl.full_bytes_per_launch
         peak = hbm
         peak_name = f"{peak_src} HBM copy bandwidth"
+    elif args.shard == "heads":
+        wl = SwaPrefill16k(hs, heads=hs.hswa_shard_kv_heads(8, ws, rank), gather_o=args.gather_o)
+        dominant_flops = wl.flops
+        peak = bf16
+        peak_name = f"{peak_src} bf16 burst"
     else:
         wl = SwaPrefill16k(hs, seq_offset=rank * 2)
         dominant_flops = wl.flops
@@ -980,7 +1046,8 @@ def main():
     kern_ms = sum(a.elapsed_time(b) for a, b in kern_events) / len(kern_events)
     ms_max = max_over_ranks(ms_step, ws)
     scale = 1e6 if decode else 1e9  # GB/s for the decode workload, TFLOP/s otherwise
-    value = weak_scaling_value(wl.flops, ws, ms_max, scale)
+    units_total = sum_over_ranks(wl.flops, ws)  # every rank's units (replicas: ws x one problem)
+    value = units_total / ms_max / scale
     achieved = dominant_flops / kern_ms / scale
     assert hs.hswa_pool_check_error(wl.pool) == 0
 
@@ -1002,7 +1069,7 @@ def main():
         b.record()
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, ws)
-        e2e = {"value": round(wl.flops * ws / e2e_ms / scale, 2), "unit": "GB/s" if decode else "TFLOP/s",
+        e2e = {"value": round(units_total / e2e_ms / scale, 2), "unit": "GB/s" if decode else "TFLOP/s",
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h,
                "path": ("pinned host Q and new K/V of 7 layers -> device, 7 hybrid_decode_fwd calls via the Python "
                         "binding (C ABI), O of 7 layers -> pinned host") if args.workload == "hybrid_decode" else
@@ -1052,17 +1119,22 @@ def main():
         elif decode:
             config = {"workload": wl.name, "n_seqs_per_gpu": wl.n, "sum_ctx": wl.S, "max_ctx": wl.maxL,
                       "tokens_per_seq": wl.nq, "window": wl.W, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
-                      "layers": "6 SWA (ring) + 1 full (pages)", "parallelism": f"independent batches x{ws}",
+                      "kv_format": "fp8_e4m3" if wl.fp8 else "bf16",
+                      "layers": "6 SWA (ring) + 1 full (pages)",
+                      "parallelism": (f"sequences split over {ws} ranks (length buckets, longest first onto the "
+                                      f"least-loaded rank; this rank {wl.n} sequences)" if args.shard == "seqs"
+                                      else f"independent batches x{ws}"),
                       "step": "7 hybrid_decode_fwd calls", "bytes_per_step": wl.bytes,
                       "l2": "inputs larger than L2 (tens of GB of K/V per step)"}
             kname = "hybrid_decode_fwd on the full layer (plan_kernel + decode_kernel<128,2> + merge_kernel)"
         else:
-            config = SwaPrefill16k.config(ws, wl.B, wl.N, wl.W, wl.Hq, wl.Hkv, wl.d)
+            config = SwaPrefill16k.config(ws, wl.B, wl.N, wl.W, wl.Hq, wl.Hkv, wl.d, args.shard, args.gather_o)
             kname = "prefill_kernel<128> (swa_prefill_fwd)"
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": ws,
             "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+            "scaling": "strong" if args.shard in ("heads", "seqs") else "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based normal, rounded to bf16)",
             "config": config,

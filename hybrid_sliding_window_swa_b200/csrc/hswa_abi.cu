@@ -412,6 +412,8 @@ int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_b
     set_error("swa_prefill_fwd: seq_ids are required with start_pos");
     return HSWA_ERR_INVALID_ARG;
   }
+  if (D.window == 1)  // the window is the diagonal alone: o_i = v_i
+    return launch_window1(pool, v, o, B, n_q, n_q_heads, D.n_kv_heads, D.head_dim, static_cast<cudaStream_t>(stream));
   PrefillLaunch L{};
   L.B = B;
   L.n_q = n_q;

@@ -60,6 +60,10 @@ int launch_gather_ring(const hswa_pool* pool, int layer, int dst, const int32_t*
 
 int launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t stream);
 
+// Sliding window W = 1: o = v of each query head's KV head (k, q and the ring are not read).
+int launch_window1(const hswa_pool* pool, const uint16_t* v, uint16_t* o, int B, int n_q, int Hq, int Hkv, int d,
+                   cudaStream_t stream);
+
 int launch_window_safe_len(const int64_t* m, const int64_t* c, const uint32_t* valid, int W, int n_req,
                            int64_t* out, cudaStream_t stream);
 

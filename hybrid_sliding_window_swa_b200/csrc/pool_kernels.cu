@@ -165,6 +165,43 @@ int launch_gather_ring(const hswa_pool* pool, int layer, int dst, const int32_t*
   return HSWA_OK;
 }
 
+// Sliding window W = 1: row i attends only key i, whose softmax weight is exactly 1, so
+// o_i = v_i of the query head's KV head (the W = 1 special case of "formal definition",
+// eq. (5)). One thread moves 16 bytes of one (row, query head).
+template <int D>
+__global__ void __launch_bounds__(256) window1_kernel(const uint16_t* __restrict__ v, uint16_t* __restrict__ o,
+                                                      int64_t rows, int Hq, int Hkv) {
+  constexpr int PER = D / 8;
+  const int G = Hq / Hkv;
+  const int64_t total = rows * Hq * PER;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(idx % PER);
+    const int64_t rh = idx / PER;
+    const int h = (int)(rh % Hq);
+    const int64_t row = rh / Hq;  // (batch, token)
+    reinterpret_cast<uint4*>(o + rh * D)[c] =
+        __ldg(reinterpret_cast<const uint4*>(v + (row * Hkv + h / G) * D) + c);
+  }
+}
+
+int launch_window1(const hswa_pool* pool, const uint16_t* v, uint16_t* o, int B, int n_q, int Hq, int Hkv, int d,
+                   cudaStream_t stream) {
+  const int64_t rows = (int64_t)B * n_q;
+  const int64_t total = rows * Hq * (d / 8);
+  if (total == 0) return HSWA_OK;
+  const int64_t want = (total + 255) / 256;
+  const int grid = (int)(want < (int64_t)pool->sms * 16 ? want : (int64_t)pool->sms * 16);
+  if (d == 128) window1_kernel<128><<<grid, 256, 0, stream>>>(v, o, rows, Hq, Hkv);
+  else window1_kernel<64><<<grid, 256, 0, stream>>>(v, o, rows, Hq, Hkv);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("swa_prefill_fwd: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
 // One thread per request. With the ring holding positions [max(0, C-W), C):
 //  * C > W: the only resumable lengths are 0 and C (every other tail reaches a
 //    position older than C - W); C needs m >= C and all W slots valid.

@@ -1,5 +1,5 @@
 // prefill_narrow.cu -- causal sliding-window prefill for narrow windows (W <= 129), where the
-// band of every 128-row query tile lies in at most two 128-key tiles.
+// band of every 128-row query tile lies in two 128-key tiles.
 //
 // Math ("Sliding Window Attention (SWA) no riron to jisso", section "formal definition",
 // eqs. (1)-(5)): query i attends keys j in [max(0, i - W + 1), i] with weights
@@ -7,21 +7,28 @@
 // "Mistral: SWA and GQA"). Tiles outside the band are never loaded (section "sparsity:
 // Flash Attention and BlockSparse").
 //
-// Work unit = (query tile t, batch row b, KV head g). The band of tile t covers key tiles
-// t - 1 and t (relative to the chunk start; tile -1 is the rolling buffer). Both key tiles
-// are loaded once per unit and stay in shared memory while the G query heads of KV head g
-// stream through two slots: slot q takes heads g*G + q, g*G + q + 2, ...
+// Work unit = (query tile t, batch row b, KV head g). Key tiles t - 1 (the rolling buffer when it
+// lies before the chunk, zeros before position 0) and t are loaded once per unit and stay in
+// shared memory while the G query heads of KV head g stream through two slots (slot q takes heads
+// q, q + 2, ... of the group). One head is one pass over both key tiles:
+//   S = Q [K_{t-1}; K_t]^T     one N = 256 MMA chain into the slot's 256 TMEM columns;
+//   one softmax over the band  row r of the tile keeps S columns [i - W + 1 - kb0, i - kb0]
+//                              (kb0 = position of column 0), which for warp w (rows 32w .. 32w+31)
+//                              lie in 32-column chunks w .. w + 4: only those five are read, and
+//                              with W = 128 away from the sequence start the band edge is the lane
+//                              index in chunks w and w + 4 and the three between are whole;
+//   P (bf16) over S's first 128 columns, O += P [V_{t-1}; V_t] into columns 128 .. 128 + D.
+// No online rescaling (one softmax step per head) and two hand-offs per head.
 //   warps 0-3 / 4-7  softmax + epilogue of slot 0 / slot 1 (one thread per TMEM lane)
-//   warp 8           K/V producer (TMA for chunk rows and aligned ring tiles, cp.async for
-//                    the others)
-//   warp 9           MMA issuer for both slots in a fixed alternating order (one thread; the
-//                    two softmax warpgroups then take turns with the tensor core); owns TMEM
-//   warp 10          Q producer: the next head of a slot is loaded as soon as that slot's last
-//                    S MMA of the current head has read its Q tile, so the load overlaps the
-//                    slot's last softmax, P V and epilogue
+//   warp 8           K/V producer: both K tiles, then both V tiles of a unit (TMA; the rolling
+//                    buffer by TMA when W = 128 and the chunk starts on a tile boundary, else
+//                    cp.async, or a dequantizing loader for FP8 pools)
+//   warp 9           MMA issuer for both slots (S of both slots, then P V of both); owns TMEM
+//   warp 10          Q producer: a slot's next head loads as soon as its S has read the Q tile
 //   warp 11          completes the warpgroup
-// TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D); P is written over S.
-// Shared memory: Q 2 tiles, K 2 tiles, V 2 tiles, output staging 2 x 16 KB.
+// TMEM: slot q owns columns [256 q, 256 q + 256).
+// Shared memory: Q 2 tiles, K [D / 64 blocks][256 rows][128 B] (tile t - 1 then tile t, so one
+// MMA reads 256 keys), V 2 tiles, output staging 32 KB.
 #include "common.cuh"
 #include "internal.h"
 #include "prefill_tile.cuh"
@@ -31,7 +38,6 @@ namespace hswa {
 namespace {
 
 constexpr int NSLOT = 2;          // query-head slots
-constexpr int NKT = 2;            // key tiles per unit (at most)
 constexpr int NWARPS = 12;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int KV_WARP = 8;
@@ -62,34 +68,29 @@ template <int D>
 struct NLayout {
   static constexpr int BLOCK = BM * 128;         // [128 rows][64 elems] swizzled = 16 KB
   static constexpr int TILE = BLOCK * (D / 64);  // one 128 x D tile
+  static constexpr int KBLK = 2 * BLOCK;         // one 64-dim block of the 256-key K operand
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + NSLOT * TILE;
-  static constexpr int V_OFF = K_OFF + NKT * TILE;
-  static constexpr int O_OFF = V_OFF + NKT * TILE;  // 4 KB output staging per softmax warp
+  static constexpr int V_OFF = K_OFF + 2 * TILE;
+  static constexpr int O_OFF = V_OFF + 2 * TILE;  // 4 KB output staging per softmax warp
   static constexpr int BAR_OFF = O_OFF + 2 * BLOCK;
   static constexpr int BYTES = BAR_OFF + 256;
   static_assert(BYTES + 1024 <= 227 * 1024, "shared memory per CTA");
-  static constexpr int O_COL0 = 256;
+  static constexpr int O_COL = 128;  // O within a slot's TMEM columns
 };
 
 struct NBars {
   uint64_t q_full[NSLOT], q_empty[NSLOT];
-  uint64_t kv_full[NKT], kv_empty[NKT];  // K and V of one key tile land together
-  uint64_t s_full[NSLOT], p_full[NSLOT], o_full[NSLOT];
+  uint64_t k_full, k_empty, v_full, v_empty;
+  uint64_t s_full[NSLOT], p_full[NSLOT], o_full[NSLOT], o_free[NSLOT];
   uint32_t tmem_base;
 };
 
 struct NGeo {
   int t, b, g, P;
-  int i0, i1;    // first / last valid absolute query position of the tile
-  int jlo, nkt;  // first key tile (relative to the chunk start) and the number of key tiles
-  int nh[NSLOT]; // heads of each slot
+  int i0;         // absolute position of the tile's first row
+  int nh[NSLOT];  // heads of each slot
 };
-
-__device__ __forceinline__ int nwindow_lo(const NParams& p, int i) {
-  const int lo = i - p.window + 1;
-  return lo > 0 ? lo : 0;
-}
 
 __device__ __forceinline__ void make_ngeo(const NParams& p, int unit, NGeo& G) {
   const int per_t = p.B * p.Hkv;
@@ -103,14 +104,88 @@ __device__ __forceinline__ void make_ngeo(const NParams& p, int unit, NGeo& G) {
     P = 0;
   }
   G.P = (int)P;
-  const int r0 = G.t * BM;
-  const int r1 = (r0 + BM - 1 < p.n_q - 1) ? r0 + BM - 1 : p.n_q - 1;
-  G.i0 = G.P + r0;
-  G.i1 = G.P + r1;
-  G.jlo = (int)floordiv(nwindow_lo(p, G.i0) - G.P, BN);
-  G.nkt = (int)floordiv(G.i1 - G.P, BN) - G.jlo + 1;
+  G.i0 = G.P + G.t * BM;
   G.nh[0] = (p.G + 1) / 2;
   G.nh[1] = p.G / 2;
+}
+
+// ---------------------------------------------------------------- one softmax pass per head
+
+// Row r of the tile at position i keeps S columns [c_lo, c_hi] of the 256 (column c = position
+// kb0 + c); warp w's rows need chunks w .. w + 4 only. FAST: W = 128 with no window clipped at
+// position 0, where c_lo = r + 1 and c_hi = r + 128, so chunk w keeps lanes j > lane, chunk w + 4
+// keeps j <= lane and chunks w + 1 .. w + 3 are whole. P = 2^(s * sl2 - m) (bf16) goes to the
+// chunk's 16 P columns (zeros for the chunks outside the five); returns the row sum.
+template <bool FAST>
+__device__ __forceinline__ float softmax_band(uint32_t trow, uint32_t s_col, int w, float sl2, int c_lo, int c_hi) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v[160];
+  tmem_ld32_into<0>(trow + s_col + 32 * (w + 0), v);
+  tmem_ld32_into<32>(trow + s_col + 32 * (w + 1), v);
+  tmem_ld32_into<64>(trow + s_col + 32 * (w + 2), v);
+  tmem_ld32_into<96>(trow + s_col + 32 * (w + 3), v);
+  tmem_ld32_into<128>(trow + s_col + 32 * (w + 4), v);
+  tmem_wait_ld();
+  reg_fence_into<0>(v);
+  reg_fence_into<32>(v);
+  reg_fence_into<64>(v);
+  reg_fence_into<96>(v);
+  reg_fence_into<128>(v);
+  if (FAST) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j <= lane) v[j] = 0xFF800000u;
+      if (j > lane) v[128 + j] = 0xFF800000u;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 5; ++c)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int col = 32 * (w + c) + j;
+        if (col < c_lo || col > c_hi) v[32 * c + j] = 0xFF800000u;
+      }
+  }
+  float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
+#pragma unroll
+  for (int k = 2; k < 160; k += 4) {
+    m0 = fmax3(m0, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+    m1 = fmax3(m1, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+  }
+  const float mx = fmaxf(m0, m1);
+  const float moff = mx == -INFINITY ? 0.f : mx * sl2;
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t neg2 = f2_pack(-moff, -moff);
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int c = 0; c < 5; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+      const uint64_t x =
+          f2_fma(f2_pack(__uint_as_float(v[32 * c + k]), __uint_as_float(v[32 * c + k + 1])), scale2, neg2);
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      const uint64_t e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      acc[(k >> 1) & 3] = f2_add(acc[(k >> 1) & 3], e);
+      float e0, e1;
+      f2_unpack(e, e0, e1);
+      pk[k >> 1] = pack_bf16x2(e0, e1);
+    }
+    tmem_st16(trow + s_col + 16 * (w + c), pk);
+  }
+  uint32_t z[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) z[k] = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (k < w || k > w + 4) tmem_st16(trow + s_col + 16 * k, z);
+  float a0, a1, b0, b1, c0, c1, d0, d1;
+  f2_unpack(acc[0], a0, a1);
+  f2_unpack(acc[1], b0, b1);
+  f2_unpack(acc[2], c0, c1);
+  f2_unpack(acc[3], d0, d1);
+  return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
 // ---------------------------------------------------------------- K/V producer
@@ -120,54 +195,56 @@ __device__ void kv_producer(const NParams& p, uint8_t* smem, NBars* bars, const 
                             const CUtensorMap* tm_v, const CUtensorMap* tm_rk, const CUtensorMap* tm_rv) {
   using L = NLayout<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t nkv[NKT] = {0, 0};  // loads per key-tile slot (kv_empty / kv_full phase)
-  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
+  uint32_t nu = 0;  // units loaded (k_empty / v_empty phase)
+  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++nu) {
     NGeo G;
     make_ngeo(p, unit, G);
     const int seq = p.seq_ids ? p.seq_ids[G.b] : 0;
     const bool seq_ok = seq >= 0 && seq < p.max_seqs;
     const int64_t ring_row = seq_ok ? ((int64_t)seq * p.n_swa + p.ring_layer) * p.Hkv + G.g : 0;
     const bool ring_fast = p.ring_tma && (G.P % BN) == 0;
-#pragma unroll
-    for (int jj = 0; jj < NKT; ++jj) {
-      if (jj >= G.nkt) break;
-      const int j = G.jlo + jj;
-      if (!mbar_wait(&bars->kv_empty[jj], (nkv[jj] & 1) ^ 1, p.err)) return;
-      ++nkv[jj];
-      uint8_t* dk = smem + L::K_OFF + jj * L::TILE;
-      uint8_t* dv = smem + L::V_OFF + jj * L::TILE;
-      if (j >= 0) {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&bars->kv_full[jj], 2 * L::TILE);
-          for (int dh = 0; dh < D / 64; ++dh) {
-            tma_load_4d(dk + dh * L::BLOCK, tm_k, &bars->kv_full[jj], dh * 64, G.g, BN * j, G.b);
-            tma_load_4d(dv + dh * L::BLOCK, tm_v, &bars->kv_full[jj], dh * 64, G.g, BN * j, G.b);
-          }
-        }
-      } else if (ring_fast) {
-        // W is a multiple of 128 and the chunk starts on a tile boundary: the tile is one box
-        if (lane == 0) {
-          if (!seq_ok) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
-          const int slot = (G.P + BN * j) % p.window;
-          const int row = seq_ok ? (int)ring_row : -1;  // outside the map: zero fill
-          mbar_arrive_expect_tx(&bars->kv_full[jj], 2 * L::TILE);
-          for (int dh = 0; dh < D / 64; ++dh) {
-            tma_load_3d(dk + dh * L::BLOCK, tm_rk, &bars->kv_full[jj], dh * 64, slot, row);
-            tma_load_3d(dv + dh * L::BLOCK, tm_rv, &bars->kv_full[jj], dh * 64, slot, row);
-          }
-        }
-      } else {
+    const int j0 = G.t - 1;                                  // key tile t - 1 (jj = 0) and t (jj = 1)
+    const bool ring_tile = j0 < 0 && p.start_pos != nullptr;  // tile t - 1 lies in the rolling buffer
+    for (int kv = 0; kv < 2; ++kv) {
+      uint64_t* full = kv ? &bars->v_full : &bars->k_full;
+      if (!mbar_wait(kv ? &bars->v_empty : &bars->k_empty, (nu & 1) ^ 1, p.err)) return;
+      const CUtensorMap* tm = kv ? tm_v : tm_k;
+      // K: the two tiles are rows 0..127 and 128..255 of each 64-dim block; V: two separate tiles
+      const int blk_stride = kv ? L::BLOCK : L::KBLK;
+      uint8_t* dst0 = smem + (kv ? L::V_OFF : L::K_OFF);
+      uint8_t* dst1 = dst0 + (kv ? L::TILE : L::BLOCK);
+      if (ring_tile && !ring_fast) {
+        // rows of the ring one by one (zeros where the ring holds nothing), before the TMA part
         if (!seq_ok && lane == 0) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
         const int held_lo = (G.P - p.window > 0) ? G.P - p.window : 0;
         const int64_t base = ring_row * p.window * D;
-        if (p.fp8) {
-          ring_rows_fp8<D>(p.ring_k8 + base, seq_ok, held_lo, G.P, p.window, p.k_scale[G.g], dk, G.P + BN * j, lane);
-          ring_rows_fp8<D>(p.ring_v8 + base, seq_ok, held_lo, G.P, p.window, p.v_scale[G.g], dv, G.P + BN * j, lane);
-        } else {
-          ring_rows_cpasync<D>(p.ring_k + base, seq_ok, held_lo, G.P, p.window, dk, G.P + BN * j, lane);
-          ring_rows_cpasync<D>(p.ring_v + base, seq_ok, held_lo, G.P, p.window, dv, G.P + BN * j, lane);
+        if (p.fp8)
+          ring_rows_fp8<D>((kv ? p.ring_v8 : p.ring_k8) + base, seq_ok, held_lo, G.P, p.window,
+                           kv ? p.v_scale[G.g] : p.k_scale[G.g], dst0, G.P + BN * j0, lane, blk_stride);
+        else
+          ring_rows_cpasync<D>((kv ? p.ring_v : p.ring_k) + base, seq_ok, held_lo, G.P, p.window, dst0,
+                               G.P + BN * j0, lane, blk_stride);
+      }
+      if (lane == 0) {
+        const bool tile0_tma = !(ring_tile && !ring_fast);
+        mbar_arrive_expect_tx(full, (tile0_tma ? 2 : 1) * L::TILE);
+        if (tile0_tma) {
+          if (ring_tile) {
+            // W = 128 and the chunk starts on a tile boundary: the tile is one box of the ring
+            if (!seq_ok) record_error(p.err, HSWA_ERR_DEVICE_BOUNDS);
+            // a tile wholly before position 0 (P = 0) is read outside the map: zero fill
+            const int slot = (G.P + BN * j0) % p.window;
+            const int row = (seq_ok && G.P + BN * j0 >= 0) ? (int)ring_row : -1;
+            for (int dh = 0; dh < D / 64; ++dh)
+              tma_load_3d(dst0 + dh * blk_stride, kv ? tm_rv : tm_rk, full, dh * 64, slot, row);
+          } else {
+            // chunk rows (tile -1 of a chunk without a prefix lies before row 0: zero fill)
+            for (int dh = 0; dh < D / 64; ++dh)
+              tma_load_4d(dst0 + dh * blk_stride, tm, full, dh * 64, G.g, BN * j0, G.b);
+          }
         }
-        if (lane == 0) mbar_arrive(&bars->kv_full[jj]);
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_4d(dst1 + dh * blk_stride, tm, full, dh * 64, G.g, BN * G.t, G.b);
       }
       __syncwarp();
     }
@@ -188,7 +265,7 @@ __device__ void q_producer(const NParams& p, uint8_t* smem, NBars* bars, const C
 #pragma unroll
       for (int q = 0; q < NSLOT; ++q) {
         if (k >= G.nh[q]) continue;
-        // the slot's Q buffer is free once its last S MMA of the previous head has completed
+        // the slot's Q buffer is free once the S of its previous head has completed
         if (!mbar_wait(&bars->q_empty[q], (nq[q] & 1) ^ 1, p.err)) return;
         ++nq[q];
         const int h = G.g * p.G + q + 2 * k;
@@ -203,88 +280,69 @@ __device__ void q_producer(const NParams& p, uint8_t* smem, NBars* bars, const C
 
 // ---------------------------------------------------------------- MMA issuer (both slots)
 
-// One thread issues both slots' MMAs in a fixed alternating order, step by step (a step is one
-// key tile of the slots' current heads): O_q += P_q V of the slot's previous S, then the slot's
-// next S. While one slot's softmax runs, the tensor core works on the other slot's products.
+// Per head k: S of both slots (each after its Q landed and its previous O was read out), then
+// P V of both (each after its softmax). While one slot's softmax or epilogue runs, the tensor
+// core works on the other slot.
 template <int D>
 __device__ void mma_issuer(const NParams& p, uint8_t* smem, NBars* bars, uint32_t tbase) {
   using L = NLayout<D>;
-  constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false);
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, 2 * BN, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
   const uint32_t q_base = smem_u32(smem + L::Q_OFF);
   const uint32_t k_base = smem_u32(smem + L::K_OFF);
   const uint32_t v_base = smem_u32(smem + L::V_OFF);
-  uint32_t np = 0;    // bit q: p_full phase of slot q
-  uint32_t nqf = 0;   // bit q: q_full phase of slot q
-  uint32_t kvph = 0;  // bit jj: kv_full phase of key-tile slot jj
+  uint32_t nqf = 0;  // bit q: q_full phase of slot q
+  uint32_t np = 0;   // bit q: p_full phase
+  uint32_t nof = 0;  // bit q: o_free phase (the slot's previous O has been read)
+  uint32_t nu = 0;   // units (k_full / v_full phase)
 
-  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
+  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++nu) {
     NGeo G;
     make_ngeo(p, unit, G);
-    uint32_t kv_ready = 0;  // bit jj: key tile jj of this unit has landed
-    int pend_jj[NSLOT] = {-1, -1};  // key tile of a slot's S whose P V is not issued yet
-    bool pend_last[NSLOT] = {false, false};  // ... and it is the head's last key tile
-    auto drain = [&](int q) -> bool {
-      if (pend_jj[q] < 0) return true;
-      if (!mbar_wait(&bars->p_full[q], (np >> q) & 1u, p.err)) return false;
-      np ^= 1u << q;
-      tc_fence_after();
-      const int jj = pend_jj[q];
-      const uint32_t vb = v_base + jj * L::TILE;
-#pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        const uint64_t bdesc = smem_desc_sw128(vb + kk * 16 * 128, L::BLOCK, 1024);
-        umma_ts(tbase + L::O_COL0 + q * 128, tbase + q * 128 + kk * 8, bdesc, IDESC_PV,
-                (jj > 0 || kk > 0) ? 1u : 0u);
-      }
-      if (pend_last[q]) umma_commit(&bars->o_full[q]);
-      pend_jj[q] = -1;
-      return true;
-    };
+    if (!mbar_wait(&bars->k_full, nu & 1, p.err)) return;
+    tc_fence_after();
     const int nk = G.nh[0] > G.nh[1] ? G.nh[0] : G.nh[1];
     for (int k = 0; k < nk; ++k) {
-      for (int jj = 0; jj < G.nkt; ++jj) {
-        if (!((kv_ready >> jj) & 1u)) {
-          if (!mbar_wait(&bars->kv_full[jj], (kvph >> jj) & 1u, p.err)) return;
-          tc_fence_after();
-          kv_ready |= 1u << jj;
-        }
 #pragma unroll
-        for (int q = 0; q < NSLOT; ++q) {
-          // P of the slot's previous key tile lives in its S columns: that P V goes first
-          if (!drain(q)) return;
-          if (k >= G.nh[q]) continue;
-          if (jj == 0) {  // a new head of the slot: its Q tile
-            if (!mbar_wait(&bars->q_full[q], (nqf >> q) & 1u, p.err)) return;
-            nqf ^= 1u << q;
-            tc_fence_after();
-          }
-          const uint32_t qb = q_base + q * L::TILE, kb = k_base + jj * L::TILE;
+      for (int q = 0; q < NSLOT; ++q) {
+        if (k >= G.nh[q]) continue;
+        if (!mbar_wait(&bars->q_full[q], (nqf >> q) & 1u, p.err)) return;
+        nqf ^= 1u << q;
+        if (!mbar_wait(&bars->o_free[q], ((nof >> q) & 1u) ^ 1u, p.err)) return;
+        nof ^= 1u << q;
+        tc_fence_after();
+        const uint32_t qb = q_base + q * L::TILE;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::BLOCK + (kk & 3) * 32;
-            umma_ss(tbase + q * 128, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                    IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars->s_full[q]);
-          if (jj == G.nkt - 1) umma_commit(&bars->q_empty[q]);  // this head's Q tile is read
-          pend_jj[q] = jj;
-          pend_last[q] = jj == G.nkt - 1;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qoff = (kk >> 2) * L::BLOCK + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * L::KBLK + (kk & 3) * 32;
+          umma_ss(tbase + 256 * q, smem_desc_sw128(qb + qoff, 16, 1024), smem_desc_sw128(k_base + koff, 16, 1024),
+                  IDESC_S, kk > 0 ? 1u : 0u);
         }
-        // the last products on key tile jj - 1 have just been issued: the producer may refill it
-        // for the next unit while this step's work runs
-        if (k == nk - 1 && jj > 0) {
-          umma_commit(&bars->kv_empty[jj - 1]);
-          kvph ^= 1u << (jj - 1);
+        umma_commit(&bars->s_full[q]);
+        umma_commit(&bars->q_empty[q]);  // this head's Q tile is read
+      }
+      if (k == nk - 1) umma_commit(&bars->k_empty);  // every S of the unit is issued
+      if (k == 0) {
+        if (!mbar_wait(&bars->v_full, nu & 1, p.err)) return;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int q = 0; q < NSLOT; ++q) {
+        if (k >= G.nh[q]) continue;
+        if (!mbar_wait(&bars->p_full[q], (np >> q) & 1u, p.err)) return;
+        np ^= 1u << q;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 2 * BN / 16; ++kk) {
+          const uint64_t bdesc =
+              smem_desc_sw128(v_base + (kk >> 3) * L::TILE + (kk & 7) * 16 * 128, L::BLOCK, 1024);
+          umma_ts(tbase + 256 * q + L::O_COL, tbase + 256 * q + kk * 8, bdesc, IDESC_PV, kk > 0 ? 1u : 0u);
         }
+        umma_commit(&bars->o_full[q]);
       }
     }
-    // the last products read the unit's last V tile: issue them, then release that tile
-#pragma unroll
-    for (int q = 0; q < NSLOT; ++q)
-      if (!drain(q)) return;
-    umma_commit(&bars->kv_empty[G.nkt - 1]);
-    kvph ^= 1u << (G.nkt - 1);
+    umma_commit(&bars->v_empty);  // every P V of the unit is issued
   }
 }
 
@@ -298,46 +356,37 @@ __device__ void softmax_slot(const NParams& p, uint8_t* smem, NBars* bars, uint3
   const int lane = threadIdx.x & 31;
   const int r = wq * 32 + lane;
   const uint32_t trow = tbase + ((uint32_t)(wq * 32) << 16);
-  const uint32_t s_col = q * 128;
-  const uint32_t o_col = L::O_COL0 + q * 128;
+  const uint32_t s_col = 256 * q;
   const float sl2 = p.scale_log2;
   uint8_t* stage = smem + L::O_OFF + q * L::BLOCK + wq * 4096;
-  uint32_t ns = 0;  // S tiles consumed (s_full phase)
-  uint32_t no = 0;  // heads finished (o_full phase)
+  uint32_t ns = 0;  // heads whose S arrived (s_full phase)
+  uint32_t no = 0;  // heads whose O arrived (o_full phase)
 
   for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
     NGeo G;
     make_ngeo(p, unit, G);
-    const int lo_last = nwindow_lo(p, G.i1);
-    // W = 128 and no row's band clipped at the sequence start: the rotated-chunk mask applies
-    const bool w128 = p.window == 128 && G.nkt == 2 && G.i0 >= 127 && G.jlo == G.t - 1;
+    const int kb0 = G.P + BN * (G.t - 1);  // position of S column 0
     const int i = G.i0 + r;
-    const int lo_i = nwindow_lo(p, i);
+    const int lo_i = (i - p.window + 1 > 0) ? i - p.window + 1 : 0;
+    const int c_lo = lo_i - kb0, c_hi = i - kb0;
+    const bool fast = p.window == 128 && G.i0 >= 127;
     for (int k = 0; k < G.nh[q]; ++k) {
-      float m_used = -INFINITY;
-      float l = 0.f;
-      for (int jj = 0; jj < G.nkt; ++jj) {
-        if (!mbar_wait(&bars->s_full[q], ns & 1, p.err)) return;
-        ++ns;
-        tc_fence_after();
-        // columns of this row inside the band: [c_lo, c_hi] (edge tiles only)
-        const int kb = G.P + BN * (G.jlo + jj);
-        const bool edge = !(kb + BN - 1 <= G.i0 && kb >= lo_last);
-        if (w128)
-          softmax_tile<D, 2>(trow, s_col, o_col, sl2, true, 0, 0, m_used, l, jj > 0, wq, jj == 0);
-        else
-          softmax_tile<D, 0>(trow, s_col, o_col, sl2, edge, lo_i - kb, i - kb, m_used, l, jj > 0);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[q]);
-      }
+      if (!mbar_wait(&bars->s_full[q], ns & 1, p.err)) return;
+      ++ns;
+      tc_fence_after();
+      const float l = fast ? softmax_band<true>(trow, s_col, wq, sl2, c_lo, c_hi)
+                           : softmax_band<false>(trow, s_col, wq, sl2, c_lo, c_hi);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[q]);
       if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
       ++no;
       tc_fence_after();
-      store_output<D>(trow, o_col, l, stage, lane, tm_o, G.g * p.G + q + 2 * k, G.t * BM + wq * 32, G.b, p.n_q);
-      // O of this head has been read: the next head's first P V may overwrite it (ordered by
-      // this warpgroup's next p_full arrival)
+      store_output<D>(trow, s_col + L::O_COL, l, stage, lane, tm_o, G.g * p.G + q + 2 * k, G.t * BM + wq * 32, G.b,
+                      p.n_q);
+      // O has been read: the slot's next S may overwrite its columns
       tc_fence_before();
+      mbar_arrive(&bars->o_free[q]);
     }
   }
 }
@@ -362,11 +411,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->s_full[q], 1);
       mbar_init(&bars->p_full[q], 128);
       mbar_init(&bars->o_full[q], 1);
+      mbar_init(&bars->o_free[q], 128);
     }
-    for (int jj = 0; jj < NKT; ++jj) {
-      mbar_init(&bars->kv_full[jj], 1);
-      mbar_init(&bars->kv_empty[jj], 1);
-    }
+    mbar_init(&bars->k_full, 1);
+    mbar_init(&bars->k_empty, 1);
+    mbar_init(&bars->v_full, 1);
+    mbar_init(&bars->v_empty, 1);
     fence_barrier_init();
   }
   if (warp == KV_WARP && (threadIdx.x & 31) == 0) {

@@ -329,10 +329,12 @@ __device__ __forceinline__ void store_output(uint32_t trow, uint32_t o_col, floa
 // Rolling-buffer rows of one key tile with cp.async (any W and chunk start), one warp:
 // positions kb .. kb + 127 come from slot pos mod W of the ring at `ring_rows` (W rows of d),
 // rows whose position the ring does not hold ([held_lo, held_hi) holds) or a bad ring are
-// zero-filled. Layout of dst: [D / 64 blocks][128 rows][128 B], 128-byte swizzle.
+// zero-filled. Layout of dst: [D / 64 blocks][128 rows][128 B], 128-byte swizzle, consecutive
+// 64-dim blocks blk_stride bytes apart (16 KB for one tile; a tile inside a taller operand
+// leaves room for the other rows).
 template <int D>
 __device__ __forceinline__ void ring_rows_cpasync(const uint16_t* ring_rows, bool ok, int held_lo, int held_hi,
-                                                  int W, uint8_t* dst, int kb, int lane) {
+                                                  int W, uint8_t* dst, int kb, int lane, int blk_stride = BM * 128) {
   const uint32_t sdst = smem_u32(dst);
   constexpr int CH = D / 8;  // 16-byte chunks per row
   for (int idx = lane; idx < BN * CH; idx += 32) {
@@ -342,7 +344,7 @@ __device__ __forceinline__ void ring_rows_cpasync(const uint16_t* ring_rows, boo
     const bool held = ok && pos >= held_lo && pos < held_hi;
     const uint16_t* src = held ? ring_rows + (int64_t)(pos % W) * D + c * 8 : ring_rows;
     const int blk = c >> 3, cc = c & 7;
-    const uint32_t off = blk * (BM * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
+    const uint32_t off = blk * blk_stride + r * 128 + ((cc ^ (r & 7)) << 4);
     cp_async_16(sdst + off, src, held ? 16u : 0u);
   }
   cp_async_wait_all();
@@ -364,13 +366,13 @@ __device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t x, float scale
 
 // ring_rows_cpasync for a ring of FP8 E4M3 codes: the held rows are dequantized (code value times
 // `scale`) to bf16 in the tile's swizzled layout; the others are zero. One warp, plain loads
-// (eight 16-byte loads in flight per lane); the caller fences and signals as for the cp.async path.
+// (four 16-byte loads in flight per lane); the caller fences and signals as for the cp.async path.
 template <int D>
 __device__ __forceinline__ void ring_rows_fp8(const uint8_t* ring_rows, bool ok, int held_lo, int held_hi, int W,
-                                              float scale, uint8_t* dst, int kb, int lane) {
+                                              float scale, uint8_t* dst, int kb, int lane, int blk_stride = BM * 128) {
   constexpr int CH8 = D / 16;           // 16-code chunks per row
   constexpr int TOTAL = BN * CH8;       // chunks per tile
-  constexpr int BATCH = 8;
+  constexpr int BATCH = 4;
   static_assert(TOTAL % (32 * BATCH) == 0, "tile chunks");
   for (int base = 0; base < TOTAL; base += 32 * BATCH) {
     uint4 x[BATCH];
@@ -399,7 +401,7 @@ __device__ __forceinline__ void ring_rows_fp8(const uint8_t* ring_rows, bool ok,
       for (int h = 0; h < 2; ++h) {
         const int cc = 2 * c + h;
         const int blk = cc >> 3, ch = cc & 7;
-        *reinterpret_cast<uint4*>(dst + blk * (BM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(dst + blk * blk_stride + r * 128 + ((ch ^ (r & 7)) << 4)) =
             make_uint4(o[4 * h], o[4 * h + 1], o[4 * h + 2], o[4 * h + 3]);
       }
     }

@@ -158,7 +158,11 @@ HSWA_API int kv_pool_gather_ring(hswa_pool* pool, int layer, int32_t dst_seq, co
  * which must hold positions [start_pos[b] - W, start_pos[b]) as committed by
  * kv_pool_append: attention reads the ring as it was before this chunk; commit
  * the chunk with kv_pool_append afterwards. Key tiles wholly outside every
- * query's window are skipped, not masked. fp32 accumulation and softmax. */
+ * query's window are skipped, not masked. fp32 accumulation and softmax.
+ * W = 1: the window is the diagonal alone, so o_i = v_i of the query head's KV head; the call
+ * copies those rows (q, k and the ring are not read). FP8 pools: keys before start_pos come from
+ * the ring dequantized (code value times scale, rounded to bf16); the chunk's own k and v are
+ * used as given. */
 HSWA_API int swa_prefill_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k,
                     const hswa_bf16* v, hswa_bf16* o, int B, int n_q, const int64_t* start_pos,
                     const int32_t* seq_ids, int n_q_heads, void* stream);
