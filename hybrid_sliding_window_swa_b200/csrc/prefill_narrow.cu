@@ -382,11 +382,9 @@ __device__ void softmax_slot(const NParams& p, uint8_t* smem, NBars* bars, uint3
       if (!mbar_wait(&bars->o_full[q], no & 1, p.err)) return;
       ++no;
       tc_fence_after();
-      store_output<D>(trow, s_col + L::O_COL, l, stage, lane, tm_o, G.g * p.G + q + 2 * k, G.t * BM + wq * 32, G.b,
-                      p.n_q);
-      // O has been read: the slot's next S may overwrite its columns
-      tc_fence_before();
-      mbar_arrive(&bars->o_free[q]);
+      // O leaves TMEM first: the slot's next S may overwrite its columns while it is stored
+      store_output_release<D>(trow, s_col + L::O_COL, l, stage, lane, tm_o, G.g * p.G + q + 2 * k,
+                              G.t * BM + wq * 32, G.b, p.n_q, &bars->o_free[q]);
     }
   }
 }

@@ -19,9 +19,9 @@
 // tile, batch row, KV head, head pair): they need the same key tiles, so each K/V tile loaded into
 // shared memory feeds both and the two slots' work is equal. With odd G the unit is two
 // consecutive query tiles of one head. The grid is persistent (one CTA per SM) and walks the
-// units in a static round-robin, heaviest (latest query tiles) first; consecutive CTAs take the
-// heads of one KV group so their K/V tiles are shared through L2.
-//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one thread per
+// units in static rounds (serpentine: every other round from the last CTA down), in blocks of query tiles (latest first) inside which the units
+// of one (batch row, KV head) are consecutive, so the CTAs share that group's K/V tiles in L2.
+//   warps 0-3   softmax for slot 0, warps 4-7 for slot 1: one thread per
 //               row (TMEM lane); all 128 scores of a row in registers, online max/sum
 //               in the exp2 domain with lazy O rescaling, MUFU exponentials (an FMA-pipe
 //               polynomial can take a share, HSWA_POLY_PER8), P written back over S as
@@ -78,6 +78,7 @@ struct Params {
   int n_pairs;     // pairs of query tiles per (batch row, head)   (G odd)
   int n_tiles;     // query tiles per batch row                    (G even)
   int head_pairs;  // 1: a unit is one query tile of two heads of a GQA group
+  int t_block;     // unit order: query tiles (or tile pairs) per block, see unit_order
   int n_units;
   int64_t max_start;  // largest start position that keeps every position below 2^31
   int* err;
@@ -130,33 +131,51 @@ __device__ __forceinline__ int key_base(const Params& p, const Geo& G, int j) {
   return p.is_full ? BN * j : G.P + BN * j;
 }
 
+// Unit order: query tiles (pairs of tiles for odd G) are cut into blocks of t_block, latest
+// (longest causal) block first; inside a block the units of one (batch row, KV head) are
+// consecutive, latest tile first. t_block = 1 is a plain latest-tile-first order (even tail); a
+// block as long as the chunk makes all CTAs walk one group's key window together (its K/V tiles
+// stay in L2 while Q and O stream through).
+__device__ __forceinline__ void unit_order(int unit, int n_t, int n_bg, int n_in, int t_block, int& t,
+                                           int& bg, int& in) {
+  const int per_block = t_block * n_bg * n_in;
+  const int k = unit / per_block;
+  const int rem = unit - k * per_block;
+  const int len = min(t_block, n_t - k * t_block);  // only the last block is shorter
+  bg = rem / (len * n_in);
+  const int r2 = rem - bg * (len * n_in);
+  t = n_t - 1 - k * t_block - r2 / n_in;
+  in = r2 - (r2 / n_in) * n_in;
+}
+
+// The unit a CTA takes in round r of the persistent loop: rounds go through the units in order,
+// every other round from the last CTA down (serpentine), so with units sorted heaviest first each
+// CTA's total work is nearly equal.
+__device__ __forceinline__ int cta_unit(int r) {
+  const int c = (HSWA_UNIT_SERPENTINE && (r & 1)) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  return r * (int)gridDim.x + c;
+}
+
 __device__ __forceinline__ void make_geo(const Params& p, int unit, Geo& G) {
   int tq[NQT];
+  int t, bg, in;
   if (p.head_pairs) {
-    const int n_hp = p.G >> 1;
-    const int per_t = p.B * p.Hkv * n_hp;
-    const int t = p.n_tiles - 1 - unit / per_t;  // latest (longest causal) tiles first
-    int rem = unit % per_t;
-    G.b = rem / (p.Hkv * n_hp);
-    rem -= G.b * (p.Hkv * n_hp);
-    G.g = rem / n_hp;
-    const int hp = rem - G.g * n_hp;
+    unit_order(unit, p.n_tiles, p.B * p.Hkv, p.G >> 1, p.t_block, t, bg, in);
+    G.b = bg / p.Hkv;
+    G.g = bg - G.b * p.Hkv;
 #pragma unroll
     for (int q = 0; q < NQT; ++q) {
       tq[q] = t;
-      G.hq[q] = G.g * p.G + 2 * hp + q;
+      G.hq[q] = G.g * p.G + 2 * in + q;
     }
   } else {
-    const int per_pair = p.B * p.Hq;
-    const int pair = p.n_pairs - 1 - unit / per_pair;  // latest (longest causal) tiles first
-    const int rem = unit % per_pair;
-    G.b = rem / p.Hq;
-    const int h = rem % p.Hq;
-    G.g = h / p.G;
+    unit_order(unit, p.n_pairs, p.B * p.Hkv, p.G, p.t_block, t, bg, in);
+    G.b = bg / p.Hkv;
+    G.g = bg - G.b * p.Hkv;
 #pragma unroll
     for (int q = 0; q < NQT; ++q) {
-      tq[q] = pair * NQT + q;
-      G.hq[q] = h;
+      tq[q] = t * NQT + q;
+      G.hq[q] = G.g * p.G + in;
     }
   }
   int64_t P = p.start_pos ? p.start_pos[G.b] : 0;
@@ -228,7 +247,7 @@ __device__ void page_converter(const Params& p, uint8_t* smem, Bars* bars) {
   static_assert(D == 128, "FP8 page tiles are converted for head_dim 128");
   const int ct = threadIdx.x - 10 * 32;  // 0 .. 63
   int it = 0;
-  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
+  for (int rnd = 0, unit = cta_unit(0); unit < p.n_units; unit = cta_unit(++rnd)) {
     Geo G;
     make_geo(p, unit, G);
     int kmax = 0;
@@ -289,7 +308,7 @@ __device__ void producer(const Params& p, uint8_t* smem, Bars* bars, const CUten
   int it = 0;        // K/V tiles loaded so far (stage ring position)
   uint32_t uq = 0;   // units started (Q buffer phase)
   uint32_t nfix = 0; // page tiles zero-filled past the last key (v_fix phase)
-  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++uq) {
+  for (int rnd = 0, unit = cta_unit(0); unit < p.n_units; unit = cta_unit(++rnd), ++uq) {
     Geo G;
     make_geo(p, unit, G);
     // the Q buffers are free once every S MMA of the previous unit has completed
@@ -427,7 +446,7 @@ __device__ void mma_issuer(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
   uint32_t np[NQT] = {0, 0};  // P tiles consumed per query tile (p_full phase)
   int it = 0;                 // K/V tiles consumed (stage ring position)
   uint32_t uq = 0;
-  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++uq) {
+  for (int rnd = 0, unit = cta_unit(0); unit < p.n_units; unit = cta_unit(++rnd), ++uq) {
     Geo G;
     make_geo(p, unit, G);
     if (!mbar_wait(&bars->q_full, uq & 1, p.err)) return;
@@ -530,7 +549,7 @@ __device__ void softmax_wg(const Params& p, uint8_t* smem, Bars* bars, uint32_t 
   uint32_t ns = 0;  // S tiles consumed (s_full phase)
   uint32_t no = 0;  // units finished (o_full phase)
 
-  for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x) {
+  for (int rnd = 0, unit = cta_unit(0); unit < p.n_units; unit = cta_unit(++rnd)) {
     Geo G;
     make_geo(p, unit, G);
     // this warpgroup's query tile, as scalars (one code path for both warpgroups)
@@ -689,12 +708,16 @@ int launch_prefill(const PrefillLaunch& Lc, cudaStream_t stream) {
   p.n_pairs = (int)((Lc.n_q + BM * NQT - 1) / (BM * NQT));
   p.n_tiles = (int)((Lc.n_q + BM - 1) / BM);
   p.head_pairs = (p.G % 2) == 0 ? 1 : 0;
+  {
+    const int n_t = p.head_pairs ? p.n_tiles : p.n_pairs;
+    p.t_block = HSWA_UNIT_TBLOCK > 0 && HSWA_UNIT_TBLOCK < n_t ? HSWA_UNIT_TBLOCK : (n_t > 0 ? n_t : 1);
+  }
   p.max_start = 0x7fffffffLL - Lc.n_q - 2 * BN;
   p.err = pool->err;
   if (Lc.n_q == 0 || Lc.B == 0) return HSWA_OK;
   const int64_t units = p.head_pairs ? (int64_t)p.n_tiles * Lc.B * Lc.Hkv * (p.G / 2)
                                      : (int64_t)p.n_pairs * Lc.B * Lc.Hq;
-  if (units > 0x7fffffff) {
+  if (units > 0x7fffffff - 65536) {  // the unit index of every round stays below 2^31
     set_error("prefill: too many work units");
     return HSWA_ERR_UNSUPPORTED_SHAPE;
   }

@@ -21,6 +21,8 @@ constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <=
 //  HSWA_SOFTMAX_SINGLE_PASS 1: keep all 128 scores of a row in registers (one TMEM read);
 //                           0: read S twice (row maximum, then exponentials), fewer registers
 //  HSWA_SOFTMAX_REGS / HSWA_PRODUCER_REGS  setmaxnreg split (2 * 128 * a + 128 * b <= 384 * 168)
+//  HSWA_UNIT_TBLOCK         prefill unit order: query tiles per block (0: the whole chunk)
+//  HSWA_UNIT_SERPENTINE     1: CTAs take the rounds of units in alternating directions
 #ifndef HSWA_POLY_PER8
 #define HSWA_POLY_PER8 0
 #endif
@@ -28,10 +30,16 @@ constexpr float kTau = 8.0f;  // lazy rescale threshold (log2 units): P stays <=
 #define HSWA_SOFTMAX_SINGLE_PASS 1
 #endif
 #ifndef HSWA_SOFTMAX_REGS
-#define HSWA_SOFTMAX_REGS 216
+#define HSWA_SOFTMAX_REGS 208
 #endif
 #ifndef HSWA_PRODUCER_REGS
-#define HSWA_PRODUCER_REGS 72
+#define HSWA_PRODUCER_REGS 88
+#endif
+#ifndef HSWA_UNIT_TBLOCK
+#define HSWA_UNIT_TBLOCK 1
+#endif
+#ifndef HSWA_UNIT_SERPENTINE
+#define HSWA_UNIT_SERPENTINE 1
 #endif
 static_assert(2 * 128 * HSWA_SOFTMAX_REGS + 128 * HSWA_PRODUCER_REGS <= 384 * 168, "register split");
 #define HSWA_STR2(x) #x
@@ -310,6 +318,57 @@ __device__ __forceinline__ void store_output(uint32_t trow, uint32_t o_col, floa
 #pragma unroll
       for (int k = 0; k < 32; k += 2)
         pk[k >> 1] = pack_bf16x2(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int chunk = (c0 >> 3) + x;
+        *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+            make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row0 < n_q) {  // a box wholly past the chunk end is not issued
+      tma_store_4d(tm_o, stage, dh * 64, h, row0, b);
+      bulk_commit_group();
+    }
+  }
+}
+
+// store_output for a caller whose next MMA waits for O's TMEM columns: all D columns of the row
+// are read into registers first, `o_free` gets this thread's arrival (the columns may be
+// overwritten from then on), and the packing, staging and TMA stores follow.
+template <int D>
+__device__ __forceinline__ void store_output_release(uint32_t trow, uint32_t o_col, float l, uint8_t* stage, int lane,
+                                                     const CUtensorMap* tm_o, int h, int row0, int b, int n_q,
+                                                     uint64_t* o_free) {
+  uint32_t o[D];
+  tmem_ld32_into<0>(trow + o_col, o);
+  tmem_ld32_into<32>(trow + o_col + 32, o);
+  if constexpr (D == 128) {
+    tmem_ld32_into<64>(trow + o_col + 64, o);
+    tmem_ld32_into<96>(trow + o_col + 96, o);
+  }
+  tmem_wait_ld();
+  reg_fence_into<0>(o);
+  reg_fence_into<32>(o);
+  if constexpr (D == 128) {
+    reg_fence_into<64>(o);
+    reg_fence_into<96>(o);
+  }
+  tc_fence_before();
+  mbar_arrive(o_free);
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int dh = 0; dh < D / 64; ++dh) {
+    if (lane == 0) bulk_wait_read_all();  // the previous store from this buffer has read it
+    __syncwarp();
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2)
+        pk[k >> 1] = pack_bf16x2(__uint_as_float(o[dh * 64 + c0 + k]) * inv,
+                                 __uint_as_float(o[dh * 64 + c0 + k + 1]) * inv);
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
         const int chunk = (c0 >> 3) + x;
