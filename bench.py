@@ -1126,7 +1126,9 @@ def main():
                                       else f"independent batches x{ws}"),
                       "step": "7 hybrid_decode_fwd calls", "bytes_per_step": wl.bytes,
                       "l2": "inputs larger than L2 (tens of GB of K/V per step)"}
-            kname = "hybrid_decode_fwd on the full layer (plan_kernel + decode_kernel<128,2> + merge_kernel)"
+            kname = ("hybrid_decode_fwd on the full layer (plan_kernel + decode_kernel<128,2> on FP8 blocks + "
+                     "merge_kernel)" if wl.fp8
+                     else "hybrid_decode_fwd on the full layer (plan_kernel + decode_kernel<128,2> + merge_kernel)")
         else:
             config = SwaPrefill16k.config(ws, wl.B, wl.N, wl.W, wl.Hq, wl.Hkv, wl.d, args.shard, args.gather_o)
             kname = "prefill_kernel<128> (swa_prefill_fwd)"

@@ -12,7 +12,7 @@ LIB = os.path.join(HERE, "libhswa.so")
 BUILD_DIR = os.path.join(HERE, "_build")
 SOURCES = ["hswa_abi.cu", "pool_kernels.cu", "prefill_sm100.cu", "prefill_narrow.cu", "decode.cu",
            "prefix_tree.cpp", "shard.cpp"]
-HEADERS = ["common.cuh", "internal.h", "prefill_tile.cuh"]
+HEADERS = ["common.cuh", "internal.h", "prefill_tile.cuh", "decode_tc.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -19,6 +19,7 @@
 // buckets and longest first, see PlanView). Items with one split write the output directly; the
 // others write (m, l, O) partials that merge_kernel combines:
 //   o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
+#include <cstddef>
 #include <mutex>
 
 #include "common.cuh"
@@ -34,6 +35,11 @@ constexpr int NST = 3;          // pipeline stages (bf16 blocks)
 constexpr int NST8 = 6;         // pipeline stages (FP8 blocks: half the bytes, the same bytes in flight)
 #ifndef HSWA_DECODE_SPLIT
 #define HSWA_DECODE_SPLIT 8192
+#endif
+#ifndef HSWA_DECODE_TC
+// FP8 pools with head_dim 128: 0 the mma.sync kernel (default, the faster one as measured), 1 the
+// tcgen05 kernel of decode_tc.cuh for full layers, 2 for every layer
+#define HSWA_DECODE_TC 0
 #endif
 constexpr int SPLIT = HSWA_DECODE_SPLIT;  // cached keys per split (tuning parameter, multiple of KB)
 static_assert(SPLIT % 64 == 0, "splits start on page boundaries");
@@ -959,6 +965,8 @@ __global__ void __launch_bounds__(256) merge_kernel(DecParams p) {
   }
 }
 
+#include "decode_tc.cuh"
+
 // Largest split count of any sequence for these arguments.
 int64_t max_splits(int window, int64_t max_ctx_len) {
   const int64_t cached = window > 0 ? (max_ctx_len < window ? max_ctx_len : window - 1) : max_ctx_len;
@@ -980,6 +988,26 @@ int launch_t(DecParams& p, int n_items_max, int sms, size_t merge_smem, cudaStre
     if (merge_smem > 48 * 1024)
       cudaFuncSetAttribute(merge_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)merge_smem);
     merge_kernel<D><<<p.n_seqs * p.Hkv, 256, merge_smem, stream>>>(p);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("hybrid_decode_fwd: launch failed: %s", cudaGetErrorString(e));
+    return HSWA_ERR_CUDA;
+  }
+  return HSWA_OK;
+}
+
+int launch_tc(DecParams& p, int n_items_max, int sms, size_t merge_smem, cudaStream_t stream) {
+  plan_kernel<<<1, 1024, 0, stream>>>(p);
+  const int smem = TcLayout::BYTES + 1024;
+  cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int grid = sms < n_items_max ? sms : n_items_max;
+  if (grid < 1) grid = 1;
+  decode_tc_kernel<<<grid, TC_THREADS, smem, stream>>>(p);
+  if (merge_smem > 0) {
+    if (merge_smem > 48 * 1024)
+      cudaFuncSetAttribute(merge_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)merge_smem);
+    merge_kernel<128><<<p.n_seqs * p.Hkv, 256, merge_smem, stream>>>(p);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -1057,6 +1085,10 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
   const int nmax = mi > 0x7fffffff ? 0x7fffffff : (int)mi;
   const size_t msm = decode_merge_smem_bytes(p.n_seqs, p.n_qt, p.Hq, p.Hkv, p.window, p.max_ctx_len);
   const int sms = pool->sms;
+  // FP8 pools with head_dim 128: the tcgen05 kernel (full layers; sliding-window layers too with
+  // HSWA_DECODE_TC=2)
+  if (pool->fp8 && Lc.d == 128 && (HSWA_DECODE_TC >= 2 || (HSWA_DECODE_TC == 1 && p.window <= 0)))
+    return launch_tc(p, nmax, sms, msm, stream);
 #define HSWA_DEC(DD, MM, F8) launch_t<DD, MM, F8>(p, nmax, sms, msm, stream)
   if (pool->fp8) {
     if (Lc.d == 128) return p.R <= 16 ? HSWA_DEC(128, 1, true) : HSWA_DEC(128, 2, true);

@@ -17,7 +17,8 @@ Workloads ("Sliding Window Attention (SWA) no riron to jisso", section "Mistral:
   * a full layer over a paged prefix (16384 cached + 4096 chunk tokens, randomly permuted
     64-token pages), Hq=64, Hkv=8: 1024 work units, 7 per CTA;
   * the hybrid decode batch: 256 sequences, context lengths log-uniform in [1K, 256K], 4 query
-    tokens each, a W=128 ring layer and a paged full layer, Hq=64, Hkv=8.
+    tokens each, a W=128 ring layer and a paged full layer, Hq=64, Hkv=8, on a bf16 pool and on
+    an FP8 (E4M3) pool.
 """
 import math
 
@@ -105,15 +106,19 @@ def test_full_layer_paged_prefix_1024_units():
     compare(o[0, rows], ref, "full layer, 16384 + 4096 keys")
 
 
-def test_hybrid_decode_256_sequences_full_size():
+def _decode_batch(seed, kv_format=hs.HSWA_KV_BF16, k_scales=None, v_scales=None):
+    """The 256-sequence decode batch on a fresh pool (a W=128 ring layer 0, a paged full layer 1)."""
     n, nq, Hq, Hkv, d, W = 256, 4, 64, 8, 128, 128
-    seed = 3104
     u = synth.uniform_float64(seed, synth.stream_id(synth.TAG_MISC, 41), n)
     lens = torch.floor(torch.exp(math.log(1024) + u * (math.log(262144) - math.log(1024)))).to(torch.int64)
     lens[int(torch.argmax(lens))] = 262144 - nq  # the longest sequence at the top of the range
     pps = (lens + nq + 63) // 64
     total_pages = int(pps.sum())
-    pool = hs.kv_pool_create(hs.PoolDesc(1, 1, W, Hkv, d, n, total_pages))
+    pool = hs.kv_pool_create(hs.PoolDesc(1, 1, W, Hkv, d, n, total_pages, kv_format=kv_format))
+    if kv_format == hs.HSWA_KV_FP8_E4M3:
+        pool.data.fill_(0x7F)  # NaN codes wherever nothing was committed
+        for layer in (0, 1):
+            pool.set_scales(layer, k_scales, v_scales)
     perm = synth.permutation(seed, synth.stream_id(synth.TAG_MISC, 42), total_pages).to(torch.int32)
     pt = torch.zeros(n, int(pps.max()), dtype=torch.int32)
     off = 0
@@ -142,6 +147,12 @@ def test_hybrid_decode_256_sequences_full_size():
         kw = dict(seq_ids=sid) if layer == 0 else dict(page_table=pt)
         outs[layer] = hs.hybrid_decode_fwd(pool, layer, q, kn, vn, ctx, maxL, ws, **kw)
     assert hs.hswa_pool_check_error(pool) == 0
+    return lens, outs, (nq, Hq, Hkv, d, W)
+
+
+def test_hybrid_decode_256_sequences_full_size():
+    seed = 3104
+    lens, outs, (nq, Hq, Hkv, d, W) = _decode_batch(seed)
     order = torch.argsort(lens, descending=True).tolist()
     # full layer: every row of the 4 longest sequences (32 splits at 256K, merged)
     for b in order[:4]:
@@ -157,3 +168,38 @@ def test_hybrid_decode_256_sequences_full_size():
         qc = q_rows(seed, 0, b, L, nq, Hq, d)
         compare(outs[0][b], oracle.attention(qc, L + np.arange(nq), kc, vc, W, key_base=L - W + 1),
                 f"ring layer, L={L}")
+
+
+def test_hybrid_decode_256_sequences_fp8_full_size():
+    """The same batch on an FP8 (E4M3) pool, against the oracle over the values the cache holds:
+    E4M3_value(E4M3(fp32(x) / s)) * s per entry, the new tokens included (they enter as they will
+    be stored)."""
+    seed = 3105
+    u = synth.uniform_float64(seed, synth.stream_id(synth.TAG_MISC, 62, 16), 16).numpy()
+    ks = (0.25 + 2.25 * u[:8]).astype(np.float32)
+    vs = (0.25 + 2.25 * u[8:]).astype(np.float32)
+    lens, outs, (nq, Hq, Hkv, d, W) = _decode_batch(seed, hs.HSWA_KV_FP8_E4M3, ks, vs)
+    lut = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))  # the oracle's value of every code
+
+    def deq(x, scales):
+        out = np.empty(tuple(x.shape), dtype=np.float64)
+        for g in range(x.shape[1]):
+            out[:, g] = lut[oracle.e4m3_quantize(x[:, g].contiguous(), scales[g])] * np.float64(scales[g])
+        return out
+
+    order = torch.argsort(lens, descending=True).tolist()
+    # full layer: every row of the 2 longest sequences (32 and more splits merged) and 2 shorter ones
+    for b in order[:2] + order[60:61] + order[-1:]:
+        L = int(lens[b])
+        kc, vc = kv_rows(seed, 1, b, 0, L + nq, Hkv, d)
+        qc = q_rows(seed, 1, b, L, nq, Hq, d)
+        ref = oracle.attention_kv64(qc, L + np.arange(nq), deq(kc, ks), deq(vc, vs), 0)
+        compare(outs[1][b], ref, f"FP8 full layer, L={L}")
+        del kc, vc, ref
+    # ring layer: every row of 6 sequences
+    for b in order[:3] + order[-3:]:
+        L = int(lens[b])
+        kc, vc = kv_rows(seed, 0, b, L - W + 1, W - 1 + nq, Hkv, d)
+        qc = q_rows(seed, 0, b, L, nq, Hq, d)
+        ref = oracle.attention_kv64(qc, L + np.arange(nq), deq(kc, ks), deq(vc, vs), W, key_base=L - W + 1)
+        compare(outs[0][b], ref, f"FP8 ring layer, L={L}")

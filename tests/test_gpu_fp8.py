@@ -71,7 +71,7 @@ def test_append_stores_the_oracle_codes(d):
     assert (ring[0, 1, 0, 0].numpy() == 0x7E).any() or (ring[0, 1, 0, 0].numpy() == 0xFE).any()
 
 
-def _decode_case(seed, lens, n_qt, hq, hkv, d, W, kind):
+def _decode_case(seed, lens, n_qt, hq, hkv, d, W, kind, ks=None, vs=None):
     n = len(lens)
     max_ctx = max(lens)
     pps = (max_ctx + n_qt + 63) // 64
@@ -80,7 +80,8 @@ def _decode_case(seed, lens, n_qt, hq, hkv, d, W, kind):
     pool = hs.kv_pool_create(desc)
     pool.data.fill_(0x7F)  # NaN codes wherever nothing was committed
     layer = 0 if kind == "swa" else 1
-    ks, vs = _scales(seed, hkv), _scales(seed + 1, hkv)
+    ks = _scales(seed, hkv) if ks is None else ks
+    vs = _scales(seed + 1, hkv) if vs is None else vs
     pool.set_scales(layer, ks, vs)
     sid = (torch.arange(n, dtype=torch.int32) * 3 % (n + 1)).contiguous()
     pt = page_table_for(seed, n, pps, total_pages).cuda() if kind == "full" else None
@@ -122,6 +123,16 @@ def test_fp8_decode_ring(W):
 ])
 def test_fp8_decode_paged(lens, n_qt, hq, hkv, d):
     _decode_case(302, lens, n_qt, hq, hkv, d, 128, "full")
+
+
+@pytest.mark.parametrize("kind", ["full", "swa"])
+def test_fp8_decode_subnormal_codes(kind):
+    """Scales of 256 put nearly every N(0, 1) entry in E4M3's subnormal range (|x / s| < 2^-6):
+    values m 2^-9 s, m = 1 .. 7. A kernel that lost them (flushed to zero) would be off by the
+    size of O itself, far outside the tolerance."""
+    hkv = 2
+    big = np.full(hkv, 256.0, dtype=np.float32)
+    _decode_case(303, [17, 64, 300, 5000], 4, 16, hkv, 128, 128, kind, ks=big, vs=big)
 
 
 def test_fp8_pool_layout_and_scale_arguments():
