@@ -1145,7 +1145,7 @@ def main():
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s" if decode else "TFLOP/s",
                          "frac": round(achieved / peak, 3), "peak_source": peak_name,
                          ("algorithmic_bytes_per_launch" if decode else "algorithmic_flops_per_launch"): dominant_flops,
-                         "kernel_ms": round(kern_ms, 4), "traffic": stored_traffic(args.workload)},
+                         "kernel_ms": round(kern_ms, 4), "traffic": stored_traffic(args.workload + ("_fp8" if args.kv_format == "fp8" and decode else ""))},
             "parity": {"max_abs_err": max_err, "mean_abs_err": mean_err},
             "gpu_launches": wl.launches_per_step * args.steps,
             "clocks": clk,
