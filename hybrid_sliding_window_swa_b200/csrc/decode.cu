@@ -20,6 +20,7 @@
 // others write (m, l, O) partials that merge_kernel combines:
 //   o = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
 #include <cstddef>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -35,11 +36,6 @@ constexpr int NST = 3;          // pipeline stages (bf16 blocks)
 constexpr int NST8 = 6;         // pipeline stages (FP8 blocks: half the bytes, the same bytes in flight)
 #ifndef HSWA_DECODE_SPLIT
 #define HSWA_DECODE_SPLIT 8192
-#endif
-#ifndef HSWA_DECODE_TC
-// FP8 pools with head_dim 128: 0 the mma.sync kernel (default, the faster one as measured), 1 the
-// tcgen05 kernel of decode_tc.cuh for full layers, 2 for every layer
-#define HSWA_DECODE_TC 0
 #endif
 constexpr int SPLIT = HSWA_DECODE_SPLIT;  // cached keys per split (tuning parameter, multiple of KB)
 static_assert(SPLIT % 64 == 0, "splits start on page boundaries");
@@ -1085,9 +1081,14 @@ int launch_decode(const DecodeLaunch& Lc, cudaStream_t stream) {
   const int nmax = mi > 0x7fffffff ? 0x7fffffff : (int)mi;
   const size_t msm = decode_merge_smem_bytes(p.n_seqs, p.n_qt, p.Hq, p.Hkv, p.window, p.max_ctx_len);
   const int sms = pool->sms;
-  // FP8 pools with head_dim 128: the tcgen05 kernel (full layers; sliding-window layers too with
-  // HSWA_DECODE_TC=2)
-  if (pool->fp8 && Lc.d == 128 && (HSWA_DECODE_TC >= 2 || (HSWA_DECODE_TC == 1 && p.window <= 0)))
+  // FP8 pools with head_dim 128 may run the tcgen05 kernel of decode_tc.cuh instead of the mma.sync
+  // one: environment variable HSWA_DECODE_TC = 1 (full layers) or 2 (every layer), read once per
+  // process; unset or 0 keeps decode_kernel, the faster of the two as measured.
+  static const int tc_mode = [] {
+    const char* e = getenv("HSWA_DECODE_TC");
+    return e ? atoi(e) : 0;
+  }();
+  if (pool->fp8 && Lc.d == 128 && (tc_mode >= 2 || (tc_mode == 1 && p.window <= 0)))
     return launch_tc(p, nmax, sms, msm, stream);
 #define HSWA_DEC(DD, MM, F8) launch_t<DD, MM, F8>(p, nmax, sms, msm, stream)
   if (pool->fp8) {

@@ -16,8 +16,8 @@
 // (exact for every E4M3 value) in the 128-byte-swizzled K-major layout the MMAs read. The K scale
 // of the KV head folds into the softmax scale and the V scale into O, so nothing else touches the
 // tiles. The new tokens' K/V are quantized as the cache will hold them.
-// Selected at build time (HSWA_DECODE_TC = 1: full layers, 2: every layer of an FP8 pool); off by
-// default. Measured on the 256-sequence batch's full layer it takes 12-13 ms against 6.9 ms for
+// Selected at run time (environment variable HSWA_DECODE_TC = 1: full layers, 2: every layer of an
+// FP8 pool with head_dim 128); off by default. Measured on the 256-sequence batch's full layer it takes 12-13 ms against 6.9 ms for
 // decode_kernel: per 128-key block the four converter warps need ~1700 clk for K and as much for V
 // (eight E4M3 -> f16 conversions per lane per 16 rows), while decode_kernel spreads the same
 // conversions over all of its warps. Correct (the FP8 decode tests pass through it) and kept as the
