@@ -970,15 +970,27 @@ def run_reference(args, ws, rank):
 
 # ------------------------------------------------------------------ main
 
-def kernel_source_sha() -> str:
-    """Hash of the CUDA sources, to tell whether a stored ncu traffic figure still describes them."""
+# the sources each workload's dominant kernel is built from (a stored traffic figure stands while
+# they are unchanged)
+KERNEL_SOURCES = {
+    "swa_prefill_16k": ["prefill_sm100.cu", "prefill_tile.cuh", "common.cuh", "internal.h"],
+    "full_chunk_131k": ["prefill_sm100.cu", "prefill_tile.cuh", "common.cuh", "internal.h"],
+    "long_context_1m": ["prefill_sm100.cu", "prefill_tile.cuh", "common.cuh", "internal.h"],
+    "swa_chunk_131k": ["prefill_narrow.cu", "prefill_tile.cuh", "common.cuh", "internal.h"],
+    "hybrid_decode": ["decode.cu", "decode_tc.cuh", "common.cuh", "internal.h"],
+    "hybrid_decode_fp8": ["decode.cu", "decode_tc.cuh", "common.cuh", "internal.h"],
+}
+
+
+def kernel_source_sha(workload: str) -> str:
+    """Hash of the CUDA sources of a workload's dominant kernel, to tell whether a stored ncu
+    traffic figure still describes them."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hybrid_sliding_window_swa_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in KERNEL_SOURCES[workload]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -988,7 +1000,7 @@ def stored_traffic(workload: str):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             d = json.load(f).get(workload)
-        if d and d.get("source_sha") == kernel_source_sha():
+        if d and d.get("source_sha") == kernel_source_sha(workload):
             return d["dram_bytes_per_launch"]
     except Exception:
         pass
