@@ -720,7 +720,37 @@ class DecodeBatch:
         return dt, byts, done
 
 
-def secondary_results(hs, oracle_mod, hbm, bf16):
+def long_context_result(hs, oracle_mod, bf16_sus):
+    """Config 5: the 70-layer step on the final 16K chunk of a 1M-token prefill (3 warm-up steps,
+    1 timed step of ~5.6 s), with its full layers against the sustained bf16 peak."""
+    wl = LongContext1M(hs)
+    for _ in range(3):
+        wl.step()
+    torch.cuda.synchronize()
+    ev = []
+    a, b = torch.cuda.Event(True), torch.cuda.Event(True)
+    a.record()
+    wl.step(ev)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    ms_full = statistics.mean(x.elapsed_time(y) for x, y in ev)
+    assert hs.hswa_pool_check_error(wl.pool) == 0
+    fp = wl.footprint()
+    mx, mean = wl.check_sample(oracle_mod)
+    full_tf = wl.full_flops_per_launch / ms_full / 1e9
+    res = {"workload": wl.name, "metric": "prefill TFLOP/s", "unit": "TFLOP/s",
+           "value": round(wl.flops / ms / 1e9, 1), "ms": round(ms, 1),
+           "full_layer_ms": round(ms_full, 2), "full_layer_tflops": round(full_tf, 1),
+           "full_layer_frac_of_sustained_peak": round(full_tf / bf16_sus, 3),
+           "footprint_slots": fp["slots"], "expected_slots_60W_plus_10N": fp["expected_slots_60W_plus_10N"],
+           "steps": 1, "warmup": 3, "max_abs_err": mx, "mean_abs_err": mean}
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def secondary_results(hs, oracle_mod, hbm, bf16, bf16_sus=None):
     out = []
     dev = "cuda"
 
@@ -805,6 +835,9 @@ def secondary_results(hs, oracle_mod, hbm, bf16):
 
     # config 4: decode batch
     out.extend(decode_results(hs, oracle_mod, hbm))
+    # config 5: the 70-layer schedule on the last chunk of a 1M-token prefill
+    if bf16_sus is not None:
+        out.append(long_context_result(hs, oracle_mod, bf16_sus))
     return out
 
 
@@ -1170,7 +1203,7 @@ def main():
                 cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                        "sample": f"{nrows} query rows x {what}, fp64, {dt:.1f} s"}
         if not args.no_secondary and ws == 1 and not big and not decode:
-            sec = secondary_results(hs, oracle, hbm, bf16)
+            sec = secondary_results(hs, oracle, hbm, bf16, bf16_sus)
 
     if rank == 0:
         if big:
