@@ -195,7 +195,11 @@ HSWA_API int hybrid_decode_workspace_size(const hswa_pool* pool, int n_seqs, int
  *  seq_ids       device int32[n_seqs] ring rows (SWA layer)
  *  page_table    device int32[n_seqs][pt_stride] (full layer)
  *  workspace     device scratch of ws_bytes >= hybrid_decode_workspace_size(); its contents
- *                on entry do not matter; calls sharing one workspace must not overlap. */
+ *                on entry do not matter; calls sharing one workspace must not overlap.
+ * FP8 pools with head_dim 128: the environment variable HSWA_DECODE_TC, read once per process,
+ * selects a tcgen05 kernel for full layers (1) or for every layer (2) instead of the default
+ * mma.sync kernel (0 or unset); both compute the same attention (within the stated tolerance),
+ * the default is the faster one as measured. */
 HSWA_API int hybrid_decode_fwd(hswa_pool* pool, int layer, const hswa_bf16* q, const hswa_bf16* k_new,
                       const hswa_bf16* v_new, hswa_bf16* o, int n_seqs, int n_q_per_seq,
                       const int64_t* ctx_len, int64_t max_ctx_len, const int32_t* seq_ids,
