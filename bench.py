@@ -448,17 +448,24 @@ class HybridChunk131k:
     first) -- tensor-bound, its metric is useful FLOPs."""
     launches_per_step = 1
 
-    def __init__(self, hs, kind="swa", seq_offset=0, P=131072, Nc=16384, W=128, Hq=64, Hkv=8, d=128):
-        self.hs, self.kind = hs, kind
+    def __init__(self, hs, kind="swa", seq_offset=0, P=131072, Nc=16384, W=128, Hq=64, Hkv=8, d=128, fp8=False):
+        self.hs, self.kind, self.fp8 = hs, kind, fp8
         self.P, self.Nc, self.W, self.Hq, self.Hkv, self.d = P, Nc, W, Hq, Hkv, d
         self.N, self.B = Nc, 1
         self.seq = 100 + seq_offset
         self.name = ("swa_chunk16k_after_131072_W128_Hq64_Hkv8_d128" if kind == "swa" else
-                     "full_chunk16k_after_131072_paged_Hq64_Hkv8_d128")
+                     "full_chunk16k_after_131072_paged_Hq64_Hkv8_d128") + ("_fp8kv" if fp8 else "")
         dev = "cuda"
         total = P + Nc
         pages = total // 64
-        self.pool = hs.kv_pool_create(hs.PoolDesc(1, 1, W, Hkv, d, 1, pages))
+        fmt = hs.HSWA_KV_FP8_E4M3 if fp8 else hs.HSWA_KV_BF16
+        self.pool = hs.kv_pool_create(hs.PoolDesc(1, 1, W, Hkv, d, 1, pages, kv_format=fmt))
+        if fp8:
+            # per-head scales of amax / 448 for |x| <= 6, as in the decode batch
+            u = synth.uniform_float64(SEED, synth.stream_id(synth.TAG_MISC, 8, seq_offset), 4 * Hkv)
+            self.scales = (6.0 / 448.0 * (0.75 + 0.5 * u)).to(torch.float32).view(2, 2, Hkv).numpy()
+            for layer in range(2):
+                self.pool.set_scales(layer, self.scales[layer, 0], self.scales[layer, 1])
         self.sid = torch.zeros(1, dtype=torch.int32, device=dev)
         self.start = torch.tensor([P], dtype=torch.int64, device=dev)
         if kind == "swa":
@@ -468,7 +475,8 @@ class HybridChunk131k:
             self.k = gen(synth.TAG_K, 0, self.seq, P, Nc, Hkv, d, 1.0, dev)[None]
             self.v = gen(synth.TAG_V, 0, self.seq, P, Nc, Hkv, d, 1.0, dev)[None]
             self.q = gen(synth.TAG_Q, 0, self.seq, P, Nc, Hq, d, 1.0, dev)[None]
-            self.flops = (2 * Nc * Hq * d + 2 * Nc * Hkv * d + 2 * (W - 1) * Hkv * d) * 2  # bytes (metric)
+            e = 1 if fp8 else 2  # bytes per ring element
+            self.flops = (2 * Nc * Hq * d + 2 * Nc * Hkv * d) * 2 + 2 * (W - 1) * Hkv * d * e  # bytes (metric)
             self.useful_flops = 4 * d * Nc * W * Hq
         else:
             perm = synth.permutation(SEED, synth.stream_id(synth.TAG_MISC, 3), pages).to(torch.int32)
@@ -521,11 +529,30 @@ class HybridChunk131k:
         q = gen(synth.TAG_Q, 1, self.seq, P, self.Nc, Hq, d, 1.0, "cpu")[rows]
         return q, k, v, 0, 0
 
+    def _deq(self, oracle, x, layer, kv):
+        """The values an FP8 pool holds for bf16 rows x [n, Hkv, d] (the oracle's decode of every
+        code as a table, times the head's scale)."""
+        lut = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+        out = np.empty(tuple(x.shape), dtype=np.float64)
+        for g in range(self.Hkv):
+            sc = float(self.scales[layer, kv, g])
+            out[:, g] = lut[oracle.e4m3_quantize(x[:, g].contiguous(), sc)] * np.float64(sc)
+        return out
+
     def check_sample(self, oracle):
         rows = [0, 1, 127, 128, 8191, self.Nc - 1] if self.kind == "swa" else [0, 5000, self.Nc - 1]
         self.step()
         q, k, v, w, base = self._ref_rows(rows)
-        ref = oracle.attention(q, self.P + np.array(rows), k, v, w, key_base=base)
+        if self.fp8:
+            # cached keys come from the FP8 pool; an SWA chunk's own keys are used as given
+            layer = 0 if self.kind == "swa" else 1
+            n_cached = self.W - 1 if self.kind == "swa" else k.shape[0]
+            k64, v64 = k.double().numpy(), v.double().numpy()
+            k64[:n_cached] = self._deq(oracle, k[:n_cached], layer, 0)
+            v64[:n_cached] = self._deq(oracle, v[:n_cached], layer, 1)
+            ref = oracle.attention_kv64(q, self.P + np.array(rows), k64, v64, w, key_base=base)
+        else:
+            ref = oracle.attention(q, self.P + np.array(rows), k, v, w, key_base=base)
         e = np.abs(self.o[0, rows].float().cpu().double().numpy() - ref)
         return float(e.max()), float(e.mean())
 
@@ -1083,7 +1110,8 @@ def main():
     hbm, bf16, bf16_sus, peak_src = peaks()
     decode = args.workload in ("hybrid_decode", "swa_chunk_131k")  # bandwidth-bound: GB/s
     if args.workload in ("swa_chunk_131k", "full_chunk_131k"):
-        wl = HybridChunk131k(hs, kind="swa" if args.workload == "swa_chunk_131k" else "full", seq_offset=rank)
+        wl = HybridChunk131k(hs, kind="swa" if args.workload == "swa_chunk_131k" else "full", seq_offset=rank,
+                             fp8=args.kv_format == "fp8")
         dominant_flops = wl.flops
         if decode:
             peak, peak_name = hbm, f"{peak_src} HBM copy bandwidth"
@@ -1218,6 +1246,7 @@ def main():
                       "window": wl.W if wl.kind == "swa" else None, "Hq": wl.Hq, "Hkv": wl.Hkv, "head_dim": wl.d,
                       "parallelism": f"independent sequences x{ws}",
                       "step": "swa_prefill_fwd" if wl.kind == "swa" else "full_prefill_fwd (chunk appended first)",
+                      "kv_format": "fp8_e4m3" if wl.fp8 else "bf16",
                       "l2": "inputs larger than L2"}
             kname = ("prefill_narrow_kernel<128> (swa_prefill_fwd, W <= 129 path)" if wl.kind == "swa" else
                      "prefill_kernel<128> (full_prefill_fwd)")
