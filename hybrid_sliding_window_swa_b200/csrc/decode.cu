@@ -425,45 +425,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
     }
     const int32_t* pt_row = p.page_table ? p.page_table + (int64_t)s * p.pt_stride : nullptr;
 
-    // ---- stage Q rows (row = t * G + hh) into shared memory, zero rows >= R
-    if constexpr (FP8) {
-      // f16, dims of each 16-dim group in the order (0,1,4,5,8,9,12,13 | 2,3,6,7,10,11,14,15)
-      for (int idx = tid; idx < ROWS * (D / 16); idx += DEC_THREADS) {
-        const int r = idx / (D / 16), grp = idx % (D / 16);
-        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (r < p.R) {
-          const int t = r / p.G, hh = r % p.G;
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + grp * 16);
-          const uint4 x0 = src[0], x1 = src[1];
-          w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
-          w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
-        }
-        // w[i] holds dims 2i (low half) and 2i + 1 (high half) as bf16
-        uint32_t c0[4], c1[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // dims 4j, 4j+1 -> chunk 0 slot j; dims 4j+2, 4j+3 -> chunk 1 slot j
-          c0[j] = pack_f16x2_sat(__uint_as_float(w[2 * j] << 16), __uint_as_float(w[2 * j] & 0xFFFF0000u));
-          c1[j] = pack_f16x2_sat(__uint_as_float(w[2 * j + 1] << 16), __uint_as_float(w[2 * j + 1] & 0xFFFF0000u));
-        }
-        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, 2 * grp)) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
-        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, 2 * grp + 1)) =
-            make_uint4(c1[0], c1[1], c1[2], c1[3]);
-      }
-    } else {
-      for (int idx = tid; idx < ROWS * (D / 8); idx += DEC_THREADS) {
-        const int r = idx / (D / 8), ch = idx % (D / 8);
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (r < p.R) {
-          const int t = r / p.G, hh = r % p.G;
-          const uint16_t* src = p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
-          val = *reinterpret_cast<const uint4*>(src);
-        }
-        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, ch)) = val;
-      }
-    }
-
     // ---- block loader: block kb2 of this item into stage st. Each copy instruction of the CTA
     // moves CP_ROWS whole rows (contiguous in HBM within a page or a ring run).
     auto kv_off = [](int r, int c) -> uint32_t {
@@ -557,6 +518,48 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       if (st < n_blk) load_block(st, st);
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
+
+    // Q is staged while the first blocks' copies are in flight (the block loop's first barrier
+    // orders it before its first use)
+    // ---- stage Q rows (row = t * G + hh) into shared memory, zero rows >= R
+    if constexpr (FP8) {
+      // f16, dims of each 16-dim group in the order (0,1,4,5,8,9,12,13 | 2,3,6,7,10,11,14,15)
+      for (int idx = tid; idx < ROWS * (D / 16); idx += DEC_THREADS) {
+        const int r = idx / (D / 16), grp = idx % (D / 16);
+        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (r < p.R) {
+          const int t = r / p.G, hh = r % p.G;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + grp * 16);
+          const uint4 x0 = src[0], x1 = src[1];
+          w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
+          w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
+        }
+        // w[i] holds dims 2i (low half) and 2i + 1 (high half) as bf16
+        uint32_t c0[4], c1[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // dims 4j, 4j+1 -> chunk 0 slot j; dims 4j+2, 4j+3 -> chunk 1 slot j
+          c0[j] = pack_f16x2_sat(__uint_as_float(w[2 * j] << 16), __uint_as_float(w[2 * j] & 0xFFFF0000u));
+          c1[j] = pack_f16x2_sat(__uint_as_float(w[2 * j + 1] << 16), __uint_as_float(w[2 * j + 1] & 0xFFFF0000u));
+        }
+        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, 2 * grp)) = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, 2 * grp + 1)) =
+            make_uint4(c1[0], c1[1], c1[2], c1[3]);
+      }
+    } else {
+      for (int idx = tid; idx < ROWS * (D / 8); idx += DEC_THREADS) {
+        const int r = idx / (D / 8), ch = idx % (D / 8);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (r < p.R) {
+          const int t = r / p.G, hh = r % p.G;
+          const uint16_t* src = p.q + (((int64_t)s * p.n_qt + t) * p.Hq + g * p.G + hh) * D + ch * 8;
+          val = *reinterpret_cast<const uint4*>(src);
+        }
+        *reinterpret_cast<uint4*>(smem + SM::Q_OFF + sw_off<D>(r, ch)) = val;
+      }
+    }
+
 
     // per-thread row state: rows (mt*16 + lane/4) and (+8)
     float o_acc[MT][D / 8][4];
