@@ -167,3 +167,25 @@ def test_kv_head_ranges_cover_every_head_once():
         assert len({e - b for b, e in ranges}) == 1
     with pytest.raises(hs.HswaError):
         hs.hswa_shard_kv_heads(8, 3, 0)  # 8 heads do not split over 3 ranks
+
+
+def test_partition_edge_cases():
+    """No sequences; more ranks than sequences (one per rank, longest on rank 0, the rest empty);
+    zero-length contexts; and the arguments the calls refuse."""
+    import numpy as np
+    import hybrid_sliding_window_swa_b200 as hs
+    ranks, loads = hs.hswa_shard_sequences(np.zeros(0, dtype=np.int64), 4)
+    assert ranks.size == 0 and list(loads) == [0, 0, 0, 0]
+    lens = np.array([70000, 300000, 1024, 65536], dtype=np.int64)  # three length buckets
+    ranks, loads = hs.hswa_shard_sequences(lens, 6)
+    assert list(ranks) == [1, 0, 3, 2]  # placed longest first, each onto the next empty rank
+    assert list(loads) == [300000, 70000, 65536, 1024, 0, 0]
+    ranks, loads = hs.hswa_shard_sequences(np.array([0, 0, 7], dtype=np.int64), 2)
+    assert list(ranks) == [1, 1, 0] and list(loads) == [7, 0]  # the 7 first; the empty ones join the least loaded
+    with pytest.raises(hs.HswaError):
+        hs.hswa_shard_sequences(np.array([5, -1], dtype=np.int64), 2)
+    with pytest.raises(hs.HswaError):
+        hs.hswa_shard_sequences(np.array([5], dtype=np.int64), 0)
+    for hkv, m, r in [(8, 2, 2), (8, 2, -1), (8, 0, 0), (0, 1, 0)]:
+        with pytest.raises(hs.HswaError):
+            hs.hswa_shard_kv_heads(hkv, m, r)
