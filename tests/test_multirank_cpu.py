@@ -56,6 +56,13 @@ def test_reference_arm_prints_on_rank0_only():
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    # the same workload description, metric and unit as the GPU arm's line (what the two arms'
+    # ratio is computed over)
+    sys.path.insert(0, ROOT)
+    import bench
+    assert line["config"] == bench.SwaPrefill16k.config(2)  # WORLD_SIZE = 2 in this run
+    assert line["metric"] == json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
 
 
 # ---------------------------------------------------------------- the multi-GPU partition
