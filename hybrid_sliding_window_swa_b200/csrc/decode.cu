@@ -665,25 +665,47 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
       for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
+          // FP8 blocks: raw scores, the scale (> 0) applied to the row maximum and inside the
+          // exponential's FMA (max(s) * c = max(s * c) exactly, rounding being monotone; measured 2%
+          // faster there); bf16 blocks: scaled scores (the other form measured 1.6% slower there)
           float v[4];
-          // allowed offsets j (key = col_base + j) for this row: lo_j <= j < hi_j
-          int lo_j = 0, hi_j = 16;
-          if (need_mask) {
-            const int hi_pos = is_new ? min(L + p.n_qt, row_pos[mt][hf] + 1) : b;  // exclusive
-            lo_j = row_lo[mt][hf] - col_base;
-            hi_j = hi_pos - col_base;
-          }
+          if constexpr (FP8) {
+            v[0] = sacc[mt][0][hf * 2 + 0];
+            v[1] = sacc[mt][0][hf * 2 + 1];
+            v[2] = sacc[mt][1][hf * 2 + 0];
+            v[3] = sacc[mt][1][hf * 2 + 1];
+            if (need_mask) {
+              // allowed offsets j (key = col_base + j) for this row: lo_j <= j < hi_j
+              const int hi_pos = is_new ? min(L + p.n_qt, row_pos[mt][hf] + 1) : b;  // exclusive
+              const int lo_j = row_lo[mt][hf] - col_base;
+              const int hi_j = hi_pos - col_base;
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int j = nt * 8 + e;
-              const float sv = sacc[mt][nt][hf * 2 + e] * sl2;
-              v[nt * 2 + e] = (j >= lo_j && j < hi_j) ? sv : -INFINITY;
+              for (int x = 0; x < 4; ++x) {
+                const int j = (x >> 1) * 8 + (x & 1);
+                if (!(j >= lo_j && j < hi_j)) v[x] = -INFINITY;
+              }
             }
+          } else {
+            // allowed offsets j (key = col_base + j) for this row: lo_j <= j < hi_j
+            int lo_j = 0, hi_j = 16;
+            if (need_mask) {
+              const int hi_pos = is_new ? min(L + p.n_qt, row_pos[mt][hf] + 1) : b;  // exclusive
+              lo_j = row_lo[mt][hf] - col_base;
+              hi_j = hi_pos - col_base;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int j = nt * 8 + e;
+                const float sv = sacc[mt][nt][hf * 2 + e] * sl2;
+                v[nt * 2 + e] = (j >= lo_j && j < hi_j) ? sv : -INFINITY;
+              }
+          }
           float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          if constexpr (FP8) mx *= sl2;
           // lazy rescale: move the offset only when the maximum grew by more than 2^8
           if (mx > m_r[mt][hf] + 8.f) {
             const float alpha = ex2_approx(m_r[mt][hf] - mx);  // 0 when the old offset is -inf
@@ -698,7 +720,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecParams p) {
           const float moff = m_r[mt][hf] == -INFINITY ? 0.f : m_r[mt][hf];
           float pv[4];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) pv[x] = ex2_approx(v[x] - moff);
+          for (int x = 0; x < 4; ++x) pv[x] = FP8 ? ex2_approx(fmaf(v[x], sl2, -moff)) : ex2_approx(v[x] - moff);
           l_r[mt][hf] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
           // A fragment of P (16 rows x 16 keys): a0/a1 = keys 0-7 (rows r, r+8), a2/a3 = keys 8-15
           if constexpr (FP8) {
