@@ -155,6 +155,18 @@ def barrier(ws):
 
 # ------------------------------------------------------------------ workloads
 
+def fp8_values(oracle_mod, x, scales):
+    """The values an FP8 pool holds for bf16 rows x [n, Hkv, d] stored with one scale per KV head:
+    the oracle's decode of every code (as a 256-entry table) times the head's scale, which is
+    oracle.e4m3_dequantize(oracle.e4m3_quantize(.)) at table-lookup speed."""
+    lut = oracle_mod.e4m3_decode(np.arange(256, dtype=np.uint8))
+    out = np.empty(tuple(x.shape), dtype=np.float64)
+    for g in range(x.shape[1]):
+        sc = np.float32(scales[g])
+        out[:, g] = lut[oracle_mod.e4m3_quantize(x[:, g].contiguous(), float(sc))] * np.float64(sc)
+    return out
+
+
 def gen(tag, layer, seq, pos0, n, h, d, sigma, device):
     return synth.normal_bf16_rows(SEED, synth.stream_id(tag, layer, seq), pos0, n, h * d, sigma, device).view(n, h, d)
 
@@ -530,14 +542,7 @@ class HybridChunk131k:
         return q, k, v, 0, 0
 
     def _deq(self, oracle, x, layer, kv):
-        """The values an FP8 pool holds for bf16 rows x [n, Hkv, d] (the oracle's decode of every
-        code as a table, times the head's scale)."""
-        lut = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
-        out = np.empty(tuple(x.shape), dtype=np.float64)
-        for g in range(self.Hkv):
-            sc = float(self.scales[layer, kv, g])
-            out[:, g] = lut[oracle.e4m3_quantize(x[:, g].contiguous(), sc)] * np.float64(sc)
-        return out
+        return fp8_values(oracle, x, self.scales[layer, kv])
 
     def check_sample(self, oracle):
         rows = [0, 1, 127, 128, 8191, self.Nc - 1] if self.kind == "swa" else [0, 5000, self.Nc - 1]
@@ -707,12 +712,8 @@ class DecodeBatch:
             q = gen(synth.TAG_Q, layer, sq, L, nq, Hq, d, 1.0, "cpu")
             if not self.fp8:
                 return oracle.attention(q, L + np.arange(nq), k, v, window, key_base=key_base)
-            kd = np.empty(tuple(k.shape), dtype=np.float64)
-            vd = np.empty(tuple(v.shape), dtype=np.float64)
-            for g in range(Hkv):
-                ks, vs = float(self.scales[layer, 0, g]), float(self.scales[layer, 1, g])
-                kd[:, g] = oracle.e4m3_dequantize(oracle.e4m3_quantize(k[:, g].contiguous(), ks), ks)
-                vd[:, g] = oracle.e4m3_dequantize(oracle.e4m3_quantize(v[:, g].contiguous(), vs), vs)
+            kd = fp8_values(oracle, k, self.scales[layer, 0])
+            vd = fp8_values(oracle, v, self.scales[layer, 1])
             return oracle.attention_kv64(q, L + np.arange(nq), kd, vd, window, key_base=key_base)
 
         for b in [int(order[0]), int(order[1]), int(order[-1])]:
